@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the sliding-window GQA attention path on B200.
+
+One step = one pass of the whole path over synthetic Mistral-7B-shaped inputs:
+  1. one-shot prefill, B=2, N=16384, W=4096, 32 query / 8 KV heads, D=128
+     (1% of key rows scaled x8) -- the headline workload;
+  2. chunked prefill of a 16384-token prompt in 4 chunks of 4096 through a
+     4096-slot rolling buffer (attention + buffer write per chunk), B=1;
+  3. batched decode: 128 steps of (append one token, attend) for B=64
+     sequences at positions drawn from [1, 32768], replayed as one CUDA graph.
+`value` is the useful (unmasked) prefill TFLOP/s of part 1; parts 2 and 3
+are reported beside it.  Inputs (0.4 GB prefill, 1 GB decode cache) are larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs the same
+independent workload (the path has no exchange step: replicas, weak
+scaling); times are the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this path
+has) on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SWA prefill useful TFLOP/s @N=16K,W=4K; decode tokens/s @B=64 (frac. of roofline)"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("device_common.cuh", "prefill_kernel.cuh", "decode_kernel.cuh", "swa_api.cu"):
+        h.update(open(os.path.join(ROOT, "sliding_window_gqa_prefill_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks sampler
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"swa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        smax = max(r["smax"] for r in rows)
+        load = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------- distributed helpers
+
+def dist_setup(gpus: int):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+_ORACLE_CACHE = {}
+
+
+def cpu_oracle_sample(target_s: float):
+    """Time the fp64 oracle on a row sample of the headline prefill workload.
+
+    Returns (TFLOP/s, seconds, rows, threads)."""
+    import numpy as np
+    import oracle
+    from sliding_window_gqa_prefill_b200 import workloads as wl
+    w = wl.HEADLINE_PREFILL
+    if "inputs" not in _ORACLE_CACHE:
+        q, k, v = wl.prefill_inputs(w)
+        _ORACLE_CACHE["inputs"] = tuple(t.float().numpy().astype(np.float64) for t in (q, k, v))
+    qn, kn, vn = _ORACLE_CACHE["inputs"]
+    rng = np.random.default_rng(0)
+    # rows past the first window: each sees exactly W keys
+    pool = rng.permutation(np.arange(w.W, w.N))
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    done, t_total, used = 0, 0.0, 0
+    batch = 8
+    while t_total < target_s and used + batch <= pool.size:
+        rows = pool[used:used + batch]
+        t0 = time.perf_counter()
+        oracle.swa_prefill(qn, kn, vn, w.W, w.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        used += batch
+        done += batch
+        remaining = target_s - t_total
+        if dt > 0 and remaining > 0:
+            batch = int(min(max(8, batch * min(4.0, remaining / dt)), pool.size - used))
+            if batch <= 0:
+                break
+    flops = 4.0 * w.B * w.Hq * w.D * w.W * done
+    return flops / t_total / 1e12, t_total, done, threads
+
+
+# ---------------------------------------------------------------- native GPU run
+
+def run_native(args):
+    import torch
+    import sliding_window_gqa_prefill_b200 as swa
+    from sliding_window_gqa_prefill_b200 import workloads as wl
+
+    rank, world, local = dist_setup(args.gpus)
+    swa.build()
+    swa.lib()
+    peaks = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    # ---- inputs, resident in HBM before timing
+    hp = wl.HEADLINE_PREFILL
+    q_cpu, k_cpu, v_cpu = wl.prefill_inputs(hp)
+    q, k, v = q_cpu.to(dev), k_cpu.to(dev), v_cpu.to(dev)
+    out = torch.empty_like(q)
+    pf_flops = wl.useful_flops(hp.B, hp.N, hp.W, hp.Hq, hp.D)
+
+    cw = wl.CHUNKED_16K
+    cq, ck, cv = (t.to(dev) for t in wl.chunked_inputs(cw))
+    c_chunks = [(cq[:, s:s + cw.C].contiguous(), ck[:, s:s + cw.C].contiguous(),
+                 cv[:, s:s + cw.C].contiguous()) for s in range(0, cw.N, cw.C)]
+    c_start = [torch.full((cw.B,), s, dtype=torch.int32, device=dev) for s in range(0, cw.N, cw.C)]
+    c_kc = torch.zeros(cw.B, cw.W, cw.Hkv, cw.D, dtype=torch.bfloat16, device=dev)
+    c_vc = torch.zeros_like(c_kc)
+    c_outs = [torch.empty_like(a) for a, _, _ in c_chunks]
+    c_flops = wl.useful_flops(cw.B, cw.N, cw.W, cw.Hq, cw.D)
+
+    dw = wl.DECODE_B64
+    dd = wl.decode_inputs(dw)
+    d_kc, d_vc = dd["k_cache"].to(dev), dd["v_cache"].to(dev)
+    d_q = dd["q"].to(dev)
+    d_kn = dd["k_new"].to(dev).unsqueeze(2).contiguous()      # [steps, B, 1, Hkv, D]
+    d_vn = dd["v_new"].to(dev).unsqueeze(2).contiguous()
+    pos_table = (dd["pos0"].unsqueeze(0) + torch.arange(dw.steps, dtype=torch.int32).unsqueeze(1)).to(torch.int32)
+    d_pos = pos_table.to(dev).contiguous()                     # [steps, B]
+    d_out = torch.empty(dw.steps, dw.B, dw.Hq, dw.D, dtype=torch.bfloat16, device=dev)
+    ws_bytes = swa.swa_decode_workspace_size(dw.B, dw.Hq, dw.Hkv, dw.D, dw.W)
+    d_ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    L = torch.clamp(pos_table.to(torch.int64) + 1, max=dw.W)   # keys read per (step, sequence)
+    kv_bytes = int(L.sum().item()) * dw.Hkv * dw.D * 2 * 2     # K and V rows read, all steps
+    other_bytes = dw.steps * dw.B * (2 * dw.Hq * dw.D * 2 + 2 * 2 * dw.Hkv * dw.D * 2)  # q, out, append r+w
+
+    def decode_all():
+        for s in range(dw.steps):
+            swa.swa_cache_append(d_kn[s], d_vn[s], d_kc, d_vc, d_pos[s])
+            swa.swa_decode(d_q[s], d_kc, d_vc, d_pos[s], dw.scale, out=d_out[s], workspace=d_ws)
+
+    # ---- capture the 128 decode steps in one graph
+    decode_all()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        decode_all()
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        swa.swa_prefill(q, k, v, hp.W, hp.scale, out=out)
+        if ev:
+            ev[1].record()
+        for (a, b, c), st, o in zip(c_chunks, c_start, c_outs):
+            swa.swa_prefill_chunk(a, b, c, c_kc, c_vc, st, cw.W, cw.scale, out=o)
+        if ev:
+            ev[2].record()
+        graph.replay()
+        if ev:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert swa.swa_get_device_status() == swa.SWA_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record()
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    status = swa.swa_get_device_status()
+    pf_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    ch_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    de_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = t_start.elapsed_time(t_end)
+
+    pf_total = max_over_ranks(sum(pf_ms), world)
+    ch_total = max_over_ranks(sum(ch_ms), world)
+    de_total = max_over_ranks(sum(de_ms), world)
+    step_total = max_over_ranks(total_ms, world)
+
+    value = pf_flops * args.steps * world / (pf_total * 1e-3) / 1e12
+    pf_avg_ms = pf_total / args.steps
+    achieved = pf_flops / (pf_avg_ms * 1e-3) / 1e12
+    chunk_tflops = c_flops * args.steps * world / (ch_total * 1e-3) / 1e12
+    dec_tok_s = dw.B * dw.steps * args.steps * world / (de_total * 1e-3)
+    dec_gbs = (kv_bytes + other_bytes) / ((de_total / args.steps) * 1e-3) / 1e9
+    dec_kv_gbs = kv_bytes / ((de_total / args.steps) * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    hq, hk, hv = q_cpu.pin_memory(), k_cpu.pin_memory(), v_cpu.pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        swa.swa_prefill(dq, dk, dv, hp.W, hp.scale, out=out)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = pf_flops * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h = hout.numel() * 2
+
+    launches_per_step = 1 + len(c_chunks) * 2 + dw.steps * (2 + (1 if ws_bytes and dw.W > 512 else 0))
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            tf, secs, rows, thr = cpu_oracle_sample(args.cpu_seconds)
+            cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                   "sample": f"{rows} query rows x B={hp.B} x {hp.Hq} heads of the headline prefill "
+                             f"(each row W={hp.W} keys), fp64, {secs:.1f} s"}
+        traffic = ncu_traffic("swa_prefill_kernel<128>")
+        result = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": step_total / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": hp.name,
+                "B": hp.B, "N": hp.N, "W": hp.W, "Hq": hp.Hq, "Hkv": hp.Hkv, "D": hp.D,
+                "parallelism": f"replicas{world}" if world > 1 else "single",
+                "l2": "inputs larger than L2 (prefill q/k/v/out 640 MB, decode cache 1 GB); no flush",
+                "step": "one-shot prefill + 4-chunk prefill (N=16384) + 128 decode steps (B=64, graph)",
+            },
+            "roofline": {
+                "bound": "tensor",
+                "kernel": "swa_prefill_kernel<128>",
+                "achieved": achieved,
+                "peak": peaks["bf16"],
+                "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16"],
+                "peak_kind": f"bf16 dense burst ({peaks['source']})",
+                "frac_of_sustained": achieved / peaks["bf16_sustained"],
+                "traffic": traffic,
+                "algorithmic_flops_per_launch": pf_flops,
+            },
+            "decode": {
+                "workload": dw.name,
+                "tokens_per_s": dec_tok_s,
+                "ms_per_128_steps": de_total / args.steps,
+                "roofline": {
+                    "bound": "hbm",
+                    "achieved": dec_gbs,
+                    "achieved_kv_only": dec_kv_gbs,
+                    "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s",
+                    "frac": dec_gbs / peaks["hbm_gbs"],
+                    "frac_kv_only": dec_kv_gbs / peaks["hbm_gbs"],
+                    "bytes_per_128_steps": kv_bytes + other_bytes,
+                    "traffic": ncu_traffic("swa_decode_kernel<128,4>"),
+                },
+            },
+            "chunked": {"workload": cw.name, "tflops": chunk_tflops,
+                        "ms": ch_total / args.steps,
+                        "frac": chunk_tflops / world / peaks["bf16"]},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "device_status": status,
+        }
+        if cpu is not None:
+            result["cpu_baseline"] = cpu
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    from sliding_window_gqa_prefill_b200 import workloads as wl
+    hp = wl.HEADLINE_PREFILL
+    per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(per_step / 4)
+    vals, secs, rows_total, thr = [], 0.0, 0, 1
+    for _ in range(args.steps):
+        tf, s, rows, thr = cpu_oracle_sample(per_step)
+        vals.append(tf)
+        secs += s
+        rows_total += rows
+    value = statistics.median(vals)
+    sample = (f"{rows_total // max(1, args.steps)} query rows per step x B={hp.B} x {hp.Hq} heads of "
+              f"the headline prefill (W={hp.W} keys each), fp64 oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": secs / max(1, args.steps) * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": hp.name, "B": hp.B, "N": hp.N, "W": hp.W, "Hq": hp.Hq,
+                   "Hkv": hp.Hkv, "D": hp.D},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_native(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

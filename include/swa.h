@@ -1,0 +1,172 @@
+/*
+ * swa.h -- C ABI of libswa: causal sliding-window attention with grouped
+ * query heads over a rolling-buffer KV cache, on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow pages written about the Mistral 7B paper
+ * (arXiv:2310.06825):
+ *  - "Mistral 7B -- Sliding Window Attention" summary (irregular6612.github.io),
+ *    sections "Methods", "핵심 구성요소" and "Rolling Buffer KV Cache 동작 설명";
+ *  - review at manon006.tistory.com/118, sections 2.2, 3.2-3.4, 4.1 (Fig. 2, 3);
+ *  - "Mistral 7B: Engineering Extreme Efficiency in LLMs" (flashpapers.ai),
+ *    sections 1 (GQA), 2 (SWA equation), 3 (rolling buffer), 4 (pre-fill and
+ *    chunking).
+ *
+ * Conventions shared by every call
+ *  - Tensors are caller-owned DEVICE memory, bfloat16 (stored as uint16_t),
+ *    contiguous row-major, with the shapes given per call.  Every tensor base
+ *    address must be 16-byte aligned.  The library never allocates, frees or
+ *    retains them; it never synchronises a stream except in
+ *    swa_get_device_status().
+ *  - Positions are 0-based int32 values in DEVICE memory, so a sequence of
+ *    calls can be captured in a CUDA graph and replayed with new positions.
+ *  - Window: query position i attends to key positions j with i-W < j <= i
+ *    (W keys, itself included).  The pages print this window two ways
+ *    ("[i-W, i-1]" and "j = i-W .. i"); the reading above is the one under
+ *    which a W-slot buffer written at slot p mod W holds every key a query
+ *    needs.  swa_prefill() also accepts the other reading, i-W <= j <= i
+ *    (SWA_WINDOW_INCL_LEFT), which is the same as W+1 under the default.
+ *  - Grouped-query heads: query head h reads KV head h / (Hq / Hkv)
+ *    (contiguous groups; Mistral-7B: 32 query heads, 8 KV heads).
+ *  - Rolling buffer: the K/V of position p live in slot p mod W of a
+ *    [B, W, Hkv, D] cache; memory stays W entries whatever the length.
+ *  - Supported: D in {64, 128}; Hq % Hkv == 0; W >= 1.  Arithmetic: bf16
+ *    inputs, fp32 accumulation and softmax, bf16 outputs (round to nearest).
+ *  - Streams: every call is asynchronous on `stream` (NULL = legacy default
+ *    stream) of the current CUDA device.
+ *  - Errors: argument checks run on the host before anything is launched and
+ *    return SWA_ERR_INVALID_ARG or SWA_ERR_UNSUPPORTED with nothing enqueued.
+ *    A failed launch returns SWA_ERR_CUDA.  Kernels never trap: each bounded
+ *    wait that runs out records SWA_ERR_TIMEOUT in a device status word, the
+ *    kernel releases what it holds and returns; swa_get_device_status()
+ *    reports it.
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *swa_stream_t;
+
+typedef enum {
+    SWA_OK = 0,
+    SWA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer */
+    SWA_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels cover */
+    SWA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    SWA_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out */
+} swa_status_t;
+
+typedef enum {
+    SWA_WINDOW_EXCL_LEFT = 0, /* keys j with i-W <  j <= i (default) */
+    SWA_WINDOW_INCL_LEFT = 1  /* keys j with i-W <= j <= i */
+} swa_window_mode_t;
+
+/*
+ * swa_prefill -- one-shot sliding-window GQA attention over a whole prompt.
+ * Pages: the SWA mask of "핵심 구성요소" and the equation of section 2 of
+ * "Engineering Extreme Efficiency"; work is O(N*W) (fully masked key tiles
+ * are never visited).
+ *   q, out : [B, N, Hq, D]       k, v : [B, N, Hkv, D]
+ *   out[b,i,h,:] = sum_j softmax_j(scale * <q[b,i,h], k[b,j,g]>) v[b,j,g]
+ *   over the window of i, g = h / (Hq/Hkv).  W >= N is dense causal.
+ * window_mode: swa_window_mode_t.  scale: softmax scale, finite and > 0.
+ */
+swa_status_t swa_prefill(const void *q, const void *k, const void *v, void *out,
+                         int B, int N, int Hq, int Hkv, int D, int W,
+                         int window_mode, float scale, swa_stream_t stream);
+
+/*
+ * swa_prefill_chunk -- pre-fill one chunk of C positions through the rolling
+ * buffer.  Pages: "Pre-fill + Chunking" in "Methods" and "핵심 구성요소", the
+ * pre-fill paragraph of the rolling-buffer section, section 4.1 / Figure 3
+ * of the review, section 4 of "Engineering Extreme Efficiency".
+ *   q, out : [B, C, Hq, D]       k, v : [B, C, Hkv, D]   (this chunk)
+ *   k_cache, v_cache : [B, W, Hkv, D], read and then updated in place
+ *   start_pos : int32 [B] device array, position of the chunk's first token
+ * Query s0+t (s0 = start_pos[b]) attends to the cached positions inside its
+ * window (the cache must hold positions s0-W .. s0-1 at slot p mod W, or be
+ * empty below position 0) and causally to the chunk itself.  After the
+ * attention the chunk's K/V are written at slots (s0+t) mod W (attend first,
+ * then write: with C = W the chunk replaces every slot).  Requires C <= W.
+ */
+swa_status_t swa_prefill_chunk(const void *q, const void *k, const void *v,
+                               void *k_cache, void *v_cache,
+                               const int32_t *start_pos, void *out, int B,
+                               int C, int Hq, int Hkv, int D, int W,
+                               float scale, swa_stream_t stream);
+
+/*
+ * swa_cache_append -- rolling-buffer write.  Pages: write step of
+ * "Rolling Buffer KV Cache 동작 설명" (slot = p % W), section 3.3 of the
+ * review, section 3 of "Engineering Extreme Efficiency".
+ *   k_new, v_new : [B, T, Hkv, D]      k_cache, v_cache : [B, W, Hkv, D]
+ *   pos : int32 [B] device array, position of each sequence's first new token
+ * cache[b, (pos[b]+t) mod W] = new[b, t], bit for bit.  Requires T <= W so
+ * that no two new tokens share a slot.  Positions must be >= 0.
+ */
+swa_status_t swa_cache_append(const void *k_new, const void *v_new,
+                              void *k_cache, void *v_cache, const int32_t *pos,
+                              int B, int T, int Hkv, int D, int W,
+                              swa_stream_t stream);
+
+/*
+ * swa_decode -- one query token per sequence against the rolling buffer.
+ * Pages: read step of "Rolling Buffer KV Cache 동작 설명" (a query at p reads
+ * positions p-W+1 .. p, which may wrap around the buffer), section 3.4 of the
+ * review (decode is bound by cache reads; GQA cuts them).
+ *   q, out : [B, Hq, D]      k_cache, v_cache : [B, W, Hkv, D]
+ *   pos : int32 [B] device array, position of the new token, whose K/V must
+ *         already be in the cache (swa_cache_append first).
+ * Each sequence reads slots 0 .. min(pos[b]+1, W)-1; softmax is order-free,
+ * so the wrap needs no reordering.
+ * workspace: device scratch of at least swa_decode_workspace_size() bytes,
+ *   256-byte aligned, owned by the caller; its contents need no set-up and are
+ *   overwritten.  Calls that share a workspace must not overlap on the GPU.
+ */
+swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *pos, void *out, int B, int Hq, int Hkv,
+                        int D, int W, float scale, void *workspace,
+                        size_t workspace_bytes, swa_stream_t stream);
+
+/* Workspace bytes swa_decode needs for these sizes (0 if they are invalid). */
+size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W);
+
+/*
+ * swa_get_device_status -- synchronise `stream`, then return (and reset to
+ * SWA_OK) the device status word that kernels of this library set when a
+ * bounded wait runs out.  Returns SWA_ERR_CUDA if synchronisation fails.
+ */
+swa_status_t swa_get_device_status(swa_stream_t stream);
+
+/*
+ * swa_set_wait_limit_ns -- limit, in nanoseconds, of every device-side wait
+ * of kernels launched afterwards on the current device (default 1 s).
+ * Test hook for the timeout path; 0 makes every wait that is not already
+ * satisfied fail at once.
+ */
+swa_status_t swa_set_wait_limit_ns(unsigned long long limit_ns);
+
+/*
+ * swa_selftest_wait_timeout -- launch one block that waits on a shared-memory
+ * barrier nothing arrives on, with the current wait limit.  The wait runs out,
+ * the kernel records SWA_ERR_TIMEOUT and returns; read it with
+ * swa_get_device_status().  Exercises the timeout path without any fault.
+ */
+swa_status_t swa_selftest_wait_timeout(swa_stream_t stream);
+
+/* Human-readable name of a status code. */
+const char *swa_status_string(swa_status_t status);
+
+/* Last CUDA error code seen by the library on this thread (0 if none). */
+int swa_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

@@ -1,0 +1,202 @@
+"""Python binding of libswa: sliding-window GQA attention over a rolling-buffer
+KV cache on B200 (sm_100a).
+
+The binding only marshals arguments: it checks tensor dtype, shape, device
+and contiguity, passes device pointers and the current CUDA stream to the C
+ABI declared in ``include/swa.h``, and turns a non-OK status into an
+exception.  Every step of the computation runs in the CUDA kernels of
+``libswa.so``; there is no fallback.  PyTorch only provides device memory and
+streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+__all__ = [
+    "SwaError", "build", "lib", "swa_prefill", "swa_prefill_chunk", "swa_cache_append",
+    "swa_decode", "swa_decode_workspace_size", "swa_get_device_status", "swa_set_wait_limit_ns",
+    "swa_selftest_wait_timeout", "SWA_OK", "SWA_ERR_INVALID_ARG", "SWA_ERR_UNSUPPORTED",
+    "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_WINDOW_EXCL_LEFT", "SWA_WINDOW_INCL_LEFT",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_PKG)
+LIB_PATH = os.path.join(_PKG, "libswa.so")
+HEADER = os.path.join(_ROOT, "include", "swa.h")
+_SOURCES = [os.path.join(_PKG, "csrc", f) for f in
+            ("swa_api.cu", "device_common.cuh", "prefill_kernel.cuh", "decode_kernel.cuh")]
+
+SWA_OK, SWA_ERR_INVALID_ARG, SWA_ERR_UNSUPPORTED, SWA_ERR_CUDA, SWA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SWA_WINDOW_EXCL_LEFT, SWA_WINDOW_INCL_LEFT = 0, 1
+
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+              "-Xcompiler", "-fPIC", "-shared"]
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED", 3: "SWA_ERR_CUDA",
+                4: "SWA_ERR_TIMEOUT"}.get(status, f"status {status}")
+        extra = ""
+        if status == SWA_ERR_CUDA and _lib is not None:
+            extra = f" (cuda error {_lib.swa_last_cuda_error()})"
+        super().__init__(f"{what}: {name}{extra}")
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libswa.so for sm_100a in the package directory (nvcc)."""
+    stale = not os.path.exists(LIB_PATH) or any(
+        os.path.getmtime(s) > os.path.getmtime(LIB_PATH) for s in _SOURCES + [HEADER])
+    if force or stale:
+        tmp = LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["nvcc", *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []),
+               "-o", tmp, os.path.join(_PKG, "csrc", "swa_api.cu")]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, LIB_PATH)
+    return LIB_PATH
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libswa.so.  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libswa.so not built ({LIB_PATH}); call "
+                                   "sliding_window_gqa_prefill_b200.build()")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, f, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+            L.swa_prefill.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, st]
+            L.swa_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, st]
+            L.swa_cache_append.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, st]
+            L.swa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, ctypes.c_size_t, st]
+            L.swa_decode_workspace_size.argtypes = [i, i, i, i, i]
+            L.swa_decode_workspace_size.restype = ctypes.c_size_t
+            L.swa_get_device_status.argtypes = [st]
+            L.swa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+            L.swa_selftest_wait_timeout.argtypes = [st]
+            L.swa_status_string.argtypes = [i]
+            L.swa_status_string.restype = ctypes.c_char_p
+            L.swa_last_cuda_error.argtypes = []
+            for fn in (L.swa_prefill, L.swa_prefill_chunk, L.swa_cache_append, L.swa_decode,
+                       L.swa_get_device_status, L.swa_set_wait_limit_ns,
+                       L.swa_selftest_wait_timeout, L.swa_last_cuda_error):
+                fn.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != SWA_OK:
+        raise SwaError(status, what)
+
+
+def _stream_handle(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _bf16(t, name: str, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name}: expected bfloat16, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _i32(t, name: str, n: int):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.int32:
+        raise TypeError(f"{name}: expected an int32 CUDA tensor")
+    if not t.is_contiguous() or t.numel() != n:
+        raise ValueError(f"{name}: expected {n} contiguous int32 values")
+    return t.data_ptr()
+
+
+def swa_prefill(q, k, v, W: int, scale: float, out=None, window_mode: int = SWA_WINDOW_EXCL_LEFT,
+                stream=None):
+    """One-shot SWA prefill.  q [B,N,Hq,D], k/v [B,N,Hkv,D] bf16 -> out [B,N,Hq,D]."""
+    import torch
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().swa_prefill(_bf16(q, "q"), _bf16(k, "k", (B, N, Hkv, D)), _bf16(v, "v", (B, N, Hkv, D)),
+                             _bf16(out, "out", (B, N, Hq, D)), B, N, Hq, Hkv, D, int(W),
+                             int(window_mode), float(scale), _stream_handle(stream)), "swa_prefill")
+    return out
+
+
+def swa_prefill_chunk(q, k, v, k_cache, v_cache, start_pos, W: int, scale: float, out=None,
+                      stream=None):
+    """Chunked prefill of one chunk through the rolling buffer (updates the cache)."""
+    import torch
+    B, C, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().swa_prefill_chunk(
+        _bf16(q, "q"), _bf16(k, "k", (B, C, Hkv, D)), _bf16(v, "v", (B, C, Hkv, D)),
+        _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _i32(start_pos, "start_pos", B), _bf16(out, "out", (B, C, Hq, D)), B, C, Hq, Hkv, D, int(W),
+        float(scale), _stream_handle(stream)), "swa_prefill_chunk")
+    return out
+
+
+def swa_cache_append(k_new, v_new, k_cache, v_cache, pos, stream=None) -> None:
+    """Write k_new/v_new [B,T,Hkv,D] at slots (pos[b]+t) mod W of the caches [B,W,Hkv,D]."""
+    B, T, Hkv, D = k_new.shape
+    W = k_cache.shape[1]
+    _check(lib().swa_cache_append(
+        _bf16(k_new, "k_new"), _bf16(v_new, "v_new", (B, T, Hkv, D)),
+        _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _i32(pos, "pos", B), B, T, Hkv, D, W, _stream_handle(stream)), "swa_cache_append")
+
+
+def swa_decode_workspace_size(B: int, Hq: int, Hkv: int, D: int, W: int) -> int:
+    return int(lib().swa_decode_workspace_size(B, Hq, Hkv, D, W))
+
+
+def swa_decode(q, k_cache, v_cache, pos, scale: float, out=None, workspace=None, stream=None):
+    """Decode one token per sequence.  q [B,Hq,D]; caches [B,W,Hkv,D]; pos int32 [B]."""
+    import torch
+    B, Hq, D = q.shape
+    W, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    need = swa_decode_workspace_size(B, Hq, Hkv, D, W)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().swa_decode(
+        _bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _i32(pos, "pos", B), _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream_handle(stream)), "swa_decode")
+    return out
+
+
+def swa_get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and reset) the device status word."""
+    return int(lib().swa_get_device_status(_stream_handle(stream)))
+
+
+def swa_set_wait_limit_ns(limit_ns: int) -> None:
+    _check(lib().swa_set_wait_limit_ns(int(limit_ns)), "swa_set_wait_limit_ns")
+
+
+def swa_selftest_wait_timeout(stream=None) -> None:
+    _check(lib().swa_selftest_wait_timeout(_stream_handle(stream)), "swa_selftest_wait_timeout")

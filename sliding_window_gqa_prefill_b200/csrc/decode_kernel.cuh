@@ -1,0 +1,368 @@
+// decode_kernel.cuh -- split-KV single-token decode over the rolling buffer,
+// and the rolling-buffer append/scatter.
+//
+// Decode: one new query token per sequence b at position pos[b], whose K/V
+// were already appended at slot pos[b] mod W.  The window (pos-W, pos] is
+// exactly the slots 0 .. L-1, L = min(pos+1, W) (read step of "Rolling Buffer
+// KV Cache 동작 설명", "Mistral 7B -- Sliding Window Attention" summary).
+// Softmax over a set of keys does not depend on their order, so the wrapped
+// buffer is read front to back with no reordering.  The query heads of one
+// GQA group read each K/V row once (section 3.4 of the manon006 review: GQA
+// cuts decode's cache reads).
+//
+// Memory-bound design (CUDA cores; the contraction is 4 x D per key, far
+// below what tensor cores need to pay off):
+//  * grid (split, kv head, sequence); a block of 4 warps streams one split of
+//    up to SPLIT keys.  Each lane owns 8 consecutive d of a key row, so a
+//    key row is read by D/8 lanes with 16-byte coalesced copies.
+//  * cp.async 16-byte copies into a per-warp 4-stage shared-memory ring keep
+//    several KB per warp in flight.
+//  * per key: partial dot products for all G heads of the group, reduced
+//    across the D/8 lanes of the row by a transposing butterfly (each level
+//    halves the values a lane holds), so a key x head score costs about one
+//    shuffle.  Online softmax per head in base 2 (scale folded into q).
+//  * warps and splits are merged by log-sum-exp: in shared memory inside a
+//    block, and by swa_decode_combine_kernel across splits.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace swa {
+
+constexpr int kDecodeSplit = 512;      // keys per block
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeStages = 4;
+
+__host__ __device__ constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x >> 1); }
+
+template <int D, int G>
+struct DecodeCfg {
+    static constexpr int LPR = D / 8;                 // lanes per key row
+    static constexpr int R = 32 / LPR;                // key rows per warp-wide load
+    static constexpr int KPR = 4;                     // keys per row group per iteration
+    static constexpr int KI = R * KPR;                // keys per warp iteration
+    static constexpr int NV = KPR * G;                // partial sums per lane
+    static constexpr int TLEV = (ilog2c(NV) < ilog2c(LPR)) ? ilog2c(NV) : ilog2c(LPR);
+    static constexpr int VPL = NV >> TLEV;            // values per lane after the butterfly
+    static constexpr int STAGE_BYTES = 2 * KI * D * 2;   // K and V rows of one iteration
+    static constexpr int WARP_RING = kDecodeStages * STAGE_BYTES;
+    static constexpr int OFF_SCORE = kDecodeWarps * WARP_RING;   // per warp [KI][G] floats
+    static constexpr int OFF_MERGE = OFF_SCORE + kDecodeWarps * KI * G * 4;
+    static constexpr int MERGE_BYTES = kDecodeWarps * G * (D + 2) * 4;
+    static constexpr int SMEM_BYTES = OFF_MERGE + MERGE_BYTES;
+    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "group size 1, 2, 4 or 8");
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// Partial result of one (sequence, kv head, split): per head m (base-2 max),
+// l (sum of 2^(s-m)) and o[D] (sum of 2^(s-m) v).  Layout in the workspace:
+// ml[((b*Hkv + g)*nsplit_max + s)*G + h] = {m, l};  o[...*D + d].
+template <int D, int G>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kc,
+                  const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ pos,
+                  __nv_bfloat16 *__restrict__ out, float2 *__restrict__ ws_ml,
+                  float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2) {
+    using Cfg = DecodeCfg<D, G>;
+    constexpr int LPR = Cfg::LPR, KPR = Cfg::KPR, KI = Cfg::KI, NV = Cfg::NV;
+    constexpr int TLEV = Cfg::TLEV, VPL = Cfg::VPL;
+    extern __shared__ __align__(128) uint8_t smem[];
+
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int Hq = Hkv * G;
+    const int p = __ldg(pos + b);
+    if (p < 0) {                                    // invalid position: record, write nothing
+        if (threadIdx.x == 0 && split == 0 && g == 0) record_status(kStatusInvalid);
+        return;
+    }
+    const int L = (p >= W - 1) ? W : p + 1;
+    const int begin = split * kDecodeSplit;
+    if (begin >= L) return;
+    const int end = min(L, begin + kDecodeSplit);
+    const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = lane / LPR;             // row group of this lane
+    const int sub = lane % LPR;             // which 8 d of the row
+    const uint32_t ring = smem_addr(smem + warp * Cfg::WARP_RING);
+    float *score = reinterpret_cast<float *>(smem + Cfg::OFF_SCORE) + warp * KI * G;
+
+    // q for every head of the group, d = sub*8 .. sub*8+7, pre-scaled to base 2
+    float qf[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)b * Hq + g * G + h) * D) + sub);
+        bf16x8_to_f32(raw, qf[h]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qf[h][e] *= scale_log2;
+    }
+
+    const size_t row_stride = (size_t)Hkv * D;     // elements between consecutive slots
+    const __nv_bfloat16 *kbase = kc + ((size_t)b * W * Hkv + g) * D + sub * 8;
+    const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv + g) * D + sub * 8;
+
+    const int n_iter_total = (end - begin + KI - 1) / KI;
+    const int my_iters = (n_iter_total > warp) ? (n_iter_total - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+
+    // stage layout: K rows [KI][D] then V rows [KI][D]
+    auto issue = [&](int it_local, int stage) {
+        const int it = warp + it_local * kDecodeWarps;
+        const uint32_t st = ring + stage * Cfg::STAGE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KPR; ++kk) {
+            const int kr = row * KPR + kk;
+            const int key = min(begin + it * KI + kr, end - 1);      // clamp: always in bounds
+            const uint32_t off = (uint32_t)((kr * D + sub * 8) * 2);
+            cp_async16(st + off, kbase + (size_t)key * row_stride);
+            cp_async16(st + KI * D * 2 + off, vbase + (size_t)key * row_stride);
+        }
+    };
+
+    float m_run[G], l_run[G], o[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        m_run[h] = -INFINITY;
+        l_run[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[h][e] = 0.f;
+    }
+
+#pragma unroll
+    for (int s = 0; s < kDecodeStages - 1; ++s) {
+        if (s < my_iters) issue(s, s);
+        cp_async_commit();
+    }
+
+    // value index of v[i] after the butterfly = vbase_idx + i
+    int vidx0 = 0;
+    {
+        int half = NV;
+#pragma unroll
+        for (int lev = 0; lev < TLEV; ++lev) {
+            half >>= 1;
+            const int off = LPR >> (lev + 1);
+            if (sub & off) vidx0 += half;
+        }
+    }
+
+    for (int it_local = 0; it_local < my_iters; ++it_local) {
+        const int stage = it_local % kDecodeStages;
+        cp_async_wait<kDecodeStages - 2>();
+        __syncwarp();
+        {
+            const int nxt = it_local + kDecodeStages - 1;
+            if (nxt < my_iters) issue(nxt, nxt % kDecodeStages);
+            cp_async_commit();
+        }
+        const uint8_t *st = smem + warp * Cfg::WARP_RING + stage * Cfg::STAGE_BYTES;
+        const int it = warp + it_local * kDecodeWarps;
+        const int key_base = begin + it * KI;
+
+        // partial dot products: value index kk*G + h
+        float v[NV];
+#pragma unroll
+        for (int kk = 0; kk < KPR; ++kk) {
+            const int kr = row * KPR + kk;
+            float kf[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(st + (kr * D + sub * 8) * 2), kf);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = fmaf(qf[h][e], kf[e], acc);
+                v[kk * G + h] = acc;
+            }
+        }
+        // transposing butterfly across the LPR lanes of the row
+        {
+#pragma unroll
+            for (int lev = 0; lev < ilog2c(LPR); ++lev) {
+                const int off = LPR >> (lev + 1);
+                if (lev < TLEV) {
+                    const int half = NV >> (lev + 1);
+                    const bool upper = (sub & off) != 0;
+#pragma unroll
+                    for (int i = 0; i < NV / 2; ++i) {
+                        if (i < half) {
+                            const float send = upper ? v[i] : v[i + half];
+                            const float keep = upper ? v[i + half] : v[i];
+                            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < VPL; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
+                }
+            }
+        }
+        // scores to shared memory (one writer per value), masking keys past the split
+        if (TLEV == ilog2c(LPR) || (sub & ((LPR >> TLEV) - 1)) == 0) {
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int idx = vidx0 + i;
+                const int kk = idx / G, h = idx % G;
+                const int kr = row * KPR + kk;
+                score[kr * G + h] = (key_base + kr < end) ? v[i] : -INFINITY;
+            }
+        }
+        __syncwarp();
+        // iteration maximum per head, then lazy-free exact online update
+        float m_new[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) m_new[h] = m_run[h];
+#pragma unroll
+        for (int kr = 0; kr < KI; ++kr)
+#pragma unroll
+            for (int h = 0; h < G; ++h) m_new[h] = fmaxf(m_new[h], score[kr * G + h]);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            if (m_new[h] > m_run[h]) {
+                const float alpha = ex2_approx(m_run[h] - m_new[h]);
+                l_run[h] *= alpha;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[h][e] *= alpha;
+                m_run[h] = m_new[h];
+            }
+        }
+        // P V for the KPR keys of this lane's row
+#pragma unroll
+        for (int kk = 0; kk < KPR; ++kk) {
+            const int kr = row * KPR + kk;
+            float vf[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(st + KI * D * 2 + (kr * D + sub * 8) * 2), vf);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float pw = ex2_approx(score[kr * G + h] - m_run[h]);
+                l_run[h] += pw;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pw, vf[e], o[h][e]);
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+
+    // merge the row groups of the warp (lanes with equal sub)
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], off);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], off);
+        }
+    }
+    // merge the warps of the block in shared memory
+    float *mg = reinterpret_cast<float *>(smem + Cfg::OFF_MERGE);    // [warp][G][D+2]
+    if (row == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float *dst = mg + (warp * G + h) * (D + 2);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dst[sub * 8 + e] = o[h][e];
+            if (sub == 0) {
+                dst[D] = m_run[h];
+                dst[D + 1] = l_run[h];
+            }
+        }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int h = idx / D, d = idx % D;
+        float m = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) m = fmaxf(m, mg[(w * G + h) * (D + 2) + D]);
+        float l = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) {
+            const float *src = mg + (w * G + h) * (D + 2);
+            const float sc = (src[D] == -INFINITY) ? 0.f : ex2_approx(src[D] - m);
+            l += src[D + 1] * sc;
+            acc += src[d] * sc;
+        }
+        if (nsplit == 1) {
+            out[((size_t)b * Hq + g * G + h) * D + d] = __float2bfloat16_rn(acc / l);
+        } else {
+            const size_t slot = ((size_t)(b * Hkv + g) * nsplit_max + split) * G + h;
+            ws_o[slot * D + d] = acc;
+            if (d == 0) ws_ml[slot] = make_float2(m, l);
+        }
+    }
+}
+
+// Log-sum-exp merge of the splits of each (sequence, kv head) into bf16 out.
+template <int D, int G>
+__global__ void __launch_bounds__(128)
+swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restrict__ ws_ml,
+                          const float *__restrict__ ws_o, __nv_bfloat16 *__restrict__ out,
+                          int Hkv, int W, int nsplit_max) {
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int Hq = Hkv * G;
+    const int p = __ldg(pos + b);
+    if (p < 0) return;
+    const int L = (p >= W - 1) ? W : p + 1;
+    const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
+    if (nsplit <= 1) return;
+    const size_t base = (size_t)(b * Hkv + g) * nsplit_max;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int h = idx / D, d = idx % D;
+        float m = -INFINITY;
+        for (int s = 0; s < nsplit; ++s) m = fmaxf(m, ws_ml[(base + s) * G + h].x);
+        float l = 0.f, acc = 0.f;
+        for (int s = 0; s < nsplit; ++s) {
+            const float2 ml = ws_ml[(base + s) * G + h];
+            const float sc = ex2_approx(ml.x - m);
+            l += ml.y * sc;
+            acc += ws_o[((base + s) * G + h) * D + d] * sc;
+        }
+        out[((size_t)b * Hq + g * G + h) * D + d] = __float2bfloat16_rn(acc / l);
+    }
+}
+
+// Rolling-buffer write: cache[b, (pos[b]+t) mod W, h, :] = new[b, t, h, :],
+// 16-byte copies, grid-stride over every (b, t, h, 16-byte chunk) of K and V.
+// Write step of "Rolling Buffer KV Cache 동작 설명" (slot = p % W).
+__global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                                  uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                                  const int32_t *__restrict__ pos, int B, int T, int W,
+                                  int row_vec) {
+    // row_vec = Hkv*D*2/16 sixteen-byte vectors per (b, t) row
+    const long long total = (long long)B * T * row_vec;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int c = (int)(i % row_vec);
+        const long long bt = i / row_vec;
+        const int t = (int)(bt % T);
+        const int b = (int)(bt / T);
+        const int p0 = __ldg(pos + b);
+        if (p0 < 0) {                               // invalid position: record, skip
+            record_status(kStatusInvalid);
+            continue;
+        }
+        const long long p = (long long)p0 + t;
+        const int slot = (int)(p % W);
+        const size_t dst = ((size_t)b * W + slot) * row_vec + c;
+        k_cache[dst] = __ldg(k_new + i);
+        v_cache[dst] = __ldg(v_new + i);
+    }
+}
+
+}  // namespace swa

@@ -1,0 +1,535 @@
+// prefill_kernel.cuh -- banded sliding-window GQA attention on tcgen05 / TMEM.
+//
+// Computes, for every query row i of a prompt (one-shot) or of a chunk that
+// continues a prompt through a rolling-buffer cache (chunked pre-fill):
+//     out[i] = sum_j softmax_j(scale * q_i . k_j) v_j
+// over the keys j of the causal window i-W < j <= i.  Sources: the SWA mask
+// of section "핵심 구성요소" of the "Mistral 7B -- Sliding Window Attention"
+// summary, the SWA equation of section 2 of "Mistral 7B: Engineering Extreme
+// Efficiency in LLMs", and for the chunked form "Pre-fill + Chunking" of the
+// same summary and section 4.1 / Figure 3 of the manon006 review.
+//
+// Design (one persistent CTA per SM):
+//  * Work unit = (sequence b, KV head g, pair of query heads of group g,
+//    block of 128 query rows).  Both query heads of the pair share every K/V
+//    tile, so one TMA load of a K/V tile feeds two 128x128 MMAs.
+//  * Only key tiles that intersect the band [q0-W+1, q0+127] are visited, so
+//    work is O(N*W).  Tiles strictly inside the band skip all masking.
+//  * Warp roles (12 warps): warp 0 issues TMA loads (Q once per unit, K and V
+//    through 3- and 2-deep rings); warp 1 issues tcgen05.mma from one thread;
+//    warp 2 owns the tensor-memory allocation; warps 4-7 and 8-11 are the
+//    softmax warpgroups of query head 0 and 1 of the pair.
+//  * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 columns each.  The
+//    softmax writes P (bf16, two per column) over the first half of its S
+//    columns and the PV MMA reads A = P straight from tensor memory.
+//  * Online softmax in fp32, base-2 exponent with the scale folded in.  The
+//    running maximum used as exponent offset is raised only when the tile
+//    maximum exceeds it by more than 8 (2^8 bound on P), so the O rescale
+//    round trip through tensor memory is rare.
+//  * Chunked pre-fill: the key tiles of a unit are the cache slot tiles that
+//    hold positions inside the window of the block (one or two runs of slots
+//    modulo W), then the chunk's own tiles.  Slot s holds position
+//    s0 - age(s), age(s) = (q - s) mod W in 1..W, q = s0 mod W, so masks are
+//    computed per element only on tiles that need them.
+//  * Every wait is bounded (SWA_ERR_TIMEOUT in the status word, then the
+//    block drains its own in-flight copies / MMAs, frees tensor memory and
+//    returns).
+#pragma once
+
+#include "device_common.cuh"
+
+namespace swa {
+
+struct PrefillParams {
+    int B;            // sequences
+    int Nq;           // query rows per sequence (N, or C in chunk mode)
+    int Nk;           // rows of the main k/v tensors (== Nq)
+    int Hq, Hkv, G;   // heads, G = Hq / Hkv
+    int W;            // window (keys i-W < j <= i)
+    int npairs;       // ceil(G / 2)
+    int nqb;          // ceil(Nq / 128)
+    int num_units;    // B * Hkv * npairs * nqb
+    float scale_log2; // softmax scale * log2(e)
+    int chunk_mode;   // 1: keys also come from the rolling-buffer cache
+    const int32_t *start_pos;  // chunk mode: [B] first position of the chunk
+    __nv_bfloat16 *out;        // [B, Nq, Hq, D]
+};
+
+template <int D>
+struct PrefillCfg {
+    static constexpr int BM = 128;                 // query rows per tile
+    static constexpr int BN = 128;                 // keys per tile
+    static constexpr int NREG = D / 64;            // 64-column (128-byte) swizzle regions
+    static constexpr int REGION_BYTES = 128 * 128; // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = NREG * REGION_BYTES;
+    static constexpr int KST = 3;                  // K ring depth
+    static constexpr int VST = 2;                  // V ring depth
+    static constexpr int OFF_Q = 0;                // two Q tiles
+    static constexpr int OFF_K = 2 * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
+    // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST],
+    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain
+    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
+    static constexpr int SMEM_BYTES = OFF_MISC + 16;
+    static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-byte alignment
+    static constexpr int THREADS = 384;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0);
+    static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, 1);
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+};
+
+// Which query rows and key tiles one work unit covers.
+struct UnitPlan {
+    int b, g, pair, qb;
+    int q0;          // first query row (relative to the q tensor)
+    int s0;          // absolute position of query row 0 of the sequence (chunk start, or 0)
+    int qs;          // s0 mod W (slot the next position would take)
+    int act1;        // second query head of the pair exists
+    int nc1, c1;     // cache run 1: tiles c1 .. c1+nc1-1
+    int nc2, c2;     // cache run 2
+    int nm, m0;      // main tiles m0 .. m0+nm-1
+    int n;           // total tiles
+};
+
+__device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u) {
+    constexpr int BM = 128, BN = 128;
+    UnitPlan P;
+    const int per = p.B * p.Hkv * p.npairs;
+    P.qb = p.nqb - 1 - u / per;          // latest (heaviest) query blocks first
+    int r = u % per;
+    P.pair = r % p.npairs;
+    r /= p.npairs;
+    P.g = r % p.Hkv;
+    P.b = r / p.Hkv;
+    P.q0 = P.qb * BM;
+    P.act1 = (2 * P.pair + 1) < p.G;
+    P.nc1 = P.nc2 = 0;
+    P.c1 = P.c2 = 0;
+    if (!p.chunk_mode) {
+        P.s0 = 0;
+        P.qs = 0;
+        const int lo = max(0, P.q0 - p.W + 1);
+        const int hi = min(p.Nk - 1, P.q0 + BM - 1);
+        P.m0 = lo / BN;
+        P.nm = hi / BN - P.m0 + 1;
+    } else {
+        P.s0 = __ldg(p.start_pos + P.b);
+        if (P.s0 < 0) {                       // invalid start: record it, attend as if 0
+            record_status(kStatusInvalid);
+            P.s0 = 0;
+        }
+        P.qs = P.s0 % p.W;
+        // oldest age any row of the block still needs: age < W - q0, age <= s0
+        const int A = min(p.W - P.q0 - 1, P.s0);
+        if (A >= 1) {
+            int last1 = -1;
+            if (P.qs >= 1) {                       // slots qs-A .. qs-1 (clipped at 0)
+                const int lo1 = max(0, P.qs - A);
+                P.c1 = lo1 / BN;
+                last1 = (P.qs - 1) / BN;
+                P.nc1 = last1 - P.c1 + 1;
+            }
+            if (A > P.qs) {                        // wrapped part: slots W-(A-qs) .. W-1
+                int lo2t = (p.W - (A - P.qs)) / BN;
+                if (lo2t <= last1) lo2t = last1 + 1;
+                const int hi2t = (p.W - 1) / BN;
+                if (lo2t <= hi2t) {
+                    P.c2 = lo2t;
+                    P.nc2 = hi2t - lo2t + 1;
+                }
+            }
+        }
+        const int hi = min(p.Nk - 1, P.q0 + BM - 1);
+        P.m0 = 0;
+        P.nm = hi / BN + 1;
+    }
+    P.n = P.nc1 + P.nc2 + P.nm;
+    return P;
+}
+
+// Key tile j of a unit: source (1 = cache), first row (slot or key index),
+// and whether any element of the 128x128 tile may be masked.
+struct TileRef {
+    int cache;
+    int row0;
+    int masked;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPlan &P, int j) {
+    constexpr int BM = 128, BN = 128;
+    TileRef t;
+    if (j < P.nc1 + P.nc2) {
+        t.cache = 1;
+        const int tile = (j < P.nc1) ? (P.c1 + j) : (P.c2 + (j - P.nc1));
+        const int k0 = tile * BN;
+        t.row0 = k0;
+        const int t_last = min(P.q0 + BM - 1, p.Nq - 1);
+        const bool has_qs = (k0 <= P.qs) && (P.qs < k0 + BN);
+        const int max_age = (k0 + BN - 1 < P.qs) ? (P.qs - k0) : (p.W - (k0 - P.qs));
+        const bool clean = !has_qs && (k0 + BN <= p.W) && (max_age < p.W - t_last) &&
+                           (max_age <= P.s0);
+        t.masked = !clean;
+    } else {
+        t.cache = 0;
+        const int k0 = (P.m0 + (j - P.nc1 - P.nc2)) * BN;
+        t.row0 = k0;
+        const bool clean = (k0 + BN - 1 <= P.q0) && (k0 > P.q0 + BM - 1 - p.W) && (k0 + BN <= p.Nk);
+        t.masked = !clean;
+    }
+    return t;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_kc,
+                   const __grid_constant__ CUtensorMap tm_vc,
+                   const PrefillParams p) {
+    using Cfg = PrefillCfg<D>;
+    constexpr int BN = Cfg::BN, KST = Cfg::KST, VST = Cfg::VST;
+    constexpr int NREG = Cfg::NREG, RB = Cfg::REGION_BYTES, TB = Cfg::TILE_BYTES;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t sQ = sbase + Cfg::OFF_Q;
+    const uint32_t sK = sbase + Cfg::OFF_K;
+    const uint32_t sV = sbase + Cfg::OFF_V;
+    const uint32_t bar0 = sbase + Cfg::OFF_BAR;
+    const uint32_t bar_q_full = bar0;
+    const uint32_t bar_q_empty = bar0 + 8;
+    const uint32_t bar_k_full = bar0 + 16;                   // + 8*slot
+    const uint32_t bar_k_empty = bar_k_full + 8 * KST;
+    const uint32_t bar_v_full = bar_k_empty + 8 * KST;
+    const uint32_t bar_v_empty = bar_v_full + 8 * VST;
+    const uint32_t bar_s_full = bar_v_empty + 8 * VST;       // + 8*t
+    const uint32_t bar_p_full = bar_s_full + 16;
+    const uint32_t bar_o_full = bar_p_full + 16;
+    const uint32_t bar_drain = bar_o_full + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const unsigned long long limit = g_wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
+        for (int s = 0; s < KST; ++s) {
+            mbar_init(bar_k_full + 8 * s, 1);
+            mbar_init(bar_k_empty + 8 * s, 1);
+        }
+        for (int s = 0; s < VST; ++s) {
+            mbar_init(bar_v_full + 8 * s, 1);
+            mbar_init(bar_v_empty + 8 * s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar_s_full + 8 * t, 1);
+            mbar_init(bar_p_full + 8 * t, 4);
+            mbar_init(bar_o_full + 8 * t, 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        if (p.chunk_mode) {
+            prefetch_tensormap(&tm_kc);
+            prefetch_tensormap(&tm_vc);
+        }
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_addr(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t kc = 0, vc = 0, uc = 0;          // tiles / units issued
+            uint32_t k_cnt[KST] = {}, v_cnt[VST] = {};
+            uint32_t q_cnt = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++uc) {
+                const UnitPlan P = plan_unit(p, u);
+                const int nact = 1 + P.act1;
+                if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
+                mbar_arrive_expect_tx(bar_q_full, nact * TB);
+                for (int t = 0; t < nact; ++t) {
+                    const int h = P.g * p.G + 2 * P.pair + t;
+                    for (int r = 0; r < NREG; ++r)
+                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, P.q0, P.b);
+                }
+                ++q_cnt;
+                for (int j = 0; j < P.n; ++j) {
+                    const TileRef T = tile_ref(p, P, j);
+                    const CUtensorMap *mk = T.cache ? &tm_kc : &tm_k;
+                    const CUtensorMap *mv = T.cache ? &tm_vc : &tm_v;
+                    const uint32_t ks = kc % KST, kph = (kc / KST) & 1;
+                    if (!mbar_wait_bounded(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, limit)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar_k_full + 8 * ks, TB);
+                    for (int r = 0; r < NREG; ++r)
+                        tma_load_4d(sK + ks * TB + r * RB, mk, bar_k_full + 8 * ks, r * 64, P.g, T.row0, P.b);
+                    ++k_cnt[ks];
+                    ++kc;
+                    const uint32_t vs = vc % VST, vph = (vc / VST) & 1;
+                    if (!mbar_wait_bounded(bar_v_empty + 8 * vs, vph ^ 1, abort_flag, limit)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar_v_full + 8 * vs, TB);
+                    for (int r = 0; r < NREG; ++r)
+                        tma_load_4d(sV + vs * TB + r * RB, mv, bar_v_full + 8 * vs, r * 64, P.g, T.row0, P.b);
+                    ++v_cnt[vs];
+                    ++vc;
+                }
+            }
+            if (!ok) {
+                // let every copy this thread started land before the block exits
+                if (q_cnt) mbar_drain_bounded(bar_q_full, (q_cnt - 1) & 1, limit);
+                for (int s = 0; s < KST; ++s)
+                    if (k_cnt[s]) mbar_drain_bounded(bar_k_full + 8 * s, (k_cnt[s] - 1) & 1, limit);
+                for (int s = 0; s < VST; ++s)
+                    if (v_cnt[s]) mbar_drain_bounded(bar_v_full + 8 * s, (v_cnt[s] - 1) & 1, limit);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t kc = 0, vc = 0, uc = 0;
+            uint32_t pc[2] = {0, 0};
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++uc) {
+                const UnitPlan P = plan_unit(p, u);
+                const int n = P.n;
+                if (!mbar_wait_bounded(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
+                // S_t = Q_t K^T for key tile j, into tensor-memory columns [t*128, t*128+128)
+                auto issue_s = [&](int t, uint32_t kslot) {
+                    const uint32_t qa = sQ + t * TB, kb = sK + kslot * TB;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * RB + (kk & 3) * 32;
+                        mma_ss(tmem + t * 128, make_smem_desc(qa + off, 16, 1024),
+                               make_smem_desc(kb + off, 16, 1024), Cfg::IDESC_QK, kk > 0);
+                    }
+                };
+                // O_t (+)= P_t V, P_t read from tensor memory over S_t's columns
+                auto issue_pv = [&](int t, uint32_t vslot, bool acc) {
+                    const uint32_t vb = sV + vslot * TB;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                               make_smem_desc(vb + kk * 16 * 128, RB, 1024), Cfg::IDESC_PV,
+                               (acc || kk > 0) ? 1u : 0u);
+                    }
+                };
+                {   // prologue: S for tile 0
+                    const uint32_t ks = kc % KST, kph = (kc / KST) & 1;
+                    if (!mbar_wait_bounded(bar_k_full + 8 * ks, kph, abort_flag, limit)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_s(0, ks);
+                    mma_commit(bar_s_full);
+                    if (P.act1) {
+                        issue_s(1, ks);
+                        mma_commit(bar_s_full + 8);
+                    }
+                    mma_commit(bar_k_empty + 8 * ks);
+                    if (n == 1) mma_commit(bar_q_empty);
+                    ++kc;
+                }
+                for (int j = 0; j < n && ok; ++j) {
+                    const uint32_t vs = vc % VST, vph = (vc / VST) & 1;
+                    if (!mbar_wait_bounded(bar_v_full + 8 * vs, vph, abort_flag, limit)) { ok = false; break; }
+                    if (!mbar_wait_bounded(bar_p_full, pc[0] & 1, abort_flag, limit)) { ok = false; break; }
+                    ++pc[0];
+                    tc_fence_after();
+                    issue_pv(0, vs, j > 0);
+                    if (j == n - 1) mma_commit(bar_o_full);
+                    uint32_t ks = 0;
+                    const bool more = (j + 1 < n);
+                    if (more) {
+                        ks = kc % KST;
+                        const uint32_t kph = (kc / KST) & 1;
+                        if (!mbar_wait_bounded(bar_k_full + 8 * ks, kph, abort_flag, limit)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_s(0, ks);
+                        mma_commit(bar_s_full);
+                    }
+                    if (P.act1) {
+                        if (!mbar_wait_bounded(bar_p_full + 8, pc[1] & 1, abort_flag, limit)) { ok = false; break; }
+                        ++pc[1];
+                        tc_fence_after();
+                        issue_pv(1, vs, j > 0);
+                        if (j == n - 1) mma_commit(bar_o_full + 8);
+                    }
+                    mma_commit(bar_v_empty + 8 * vs);
+                    ++vc;
+                    if (more) {
+                        if (P.act1) {
+                            issue_s(1, ks);
+                            mma_commit(bar_s_full + 8);
+                        }
+                        mma_commit(bar_k_empty + 8 * ks);
+                        if (j + 1 == n - 1) mma_commit(bar_q_empty);
+                        ++kc;
+                    }
+                }
+            }
+            if (!ok) {
+                mma_commit(bar_drain);
+                mbar_drain_bounded(bar_drain, 0, limit);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = (warp - 4) >> 2;            // query head of the pair
+        const int quarter = warp & 3;             // TMEM lane quarter of this warp
+        const int row = quarter * 32 + lane;      // query row within the tile
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + t * 128;
+        const uint32_t tO = tmem + lane_off + 256 + t * 128;
+        const float sl2 = p.scale_log2;
+        uint32_t sc = 0, oc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const UnitPlan P = plan_unit(p, u);
+            if (t == 1 && !P.act1) continue;
+            const int i_rel = P.q0 + row;                  // query row in the q tensor
+            float m_use = -INFINITY, l = 0.f;
+            for (int j = 0; j < P.n; ++j) {
+                const TileRef T = tile_ref(p, P, j);
+                // warp-uniform outcome, so the collective tensor-memory ops stay converged
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_s_full + 8 * t, sc & 1, abort_flag, limit))) {
+                    ok = false;
+                    break;
+                }
+                ++sc;
+                tc_fence_after();
+                float s[BN];
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + c * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+                }
+                if (T.masked) {
+                    if (T.cache) {
+                        // slot k0+c holds position s0 - age; valid iff age < W - t_rel, age <= s0
+                        const int lim = min(p.W - i_rel - 1, P.s0);
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) {
+                            const int slot = T.row0 + c;
+                            const int age = (slot < P.qs) ? (P.qs - slot) : (P.qs - slot + p.W);
+                            if (slot >= p.W || age > lim) s[c] = -INFINITY;
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) {
+                            const int key = T.row0 + c;
+                            if (key > i_rel || key <= i_rel - p.W) s[c] = -INFINITY;
+                        }
+                    }
+                }
+                float mt = s[0];
+#pragma unroll
+                for (int c = 1; c < BN; ++c) mt = fmaxf(mt, s[c]);
+                const float m_tile = mt * sl2;
+                const float m_cand = fmaxf(m_use, m_tile);
+                if (j == 0) {
+                    m_use = m_cand;
+                } else {
+                    const bool need = m_cand > m_use + 8.0f;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float alpha = need ? ex2_approx(m_use - m_cand) : 1.0f;
+                        if (need) {
+                            l *= alpha;
+                            m_use = m_cand;
+                        }
+#pragma unroll 1
+                        for (int c = 0; c < D / 16; ++c) {
+                            uint32_t r[16];
+                            tmem_ld16(tO + c * 16, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st16(tO + c * 16, r);
+                        }
+                    }
+                }
+                const float mb = (m_use == -INFINITY) ? 0.f : m_use;
+                float lsum = 0.f;
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * e], sl2, -mb));
+                        const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * e + 1], sl2, -mb));
+                        lsum += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + c * 16, pk);
+                }
+                l += lsum;
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_p_full + 8 * t);
+            }
+            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_o_full + 8 * t, oc & 1, abort_flag, limit))) {
+                ok = false;
+                break;
+            }
+            ++oc;
+            tc_fence_after();
+            const int h = P.g * p.G + 2 * P.pair + t;
+            const bool valid_row = i_rel < p.Nq;
+            const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+            __nv_bfloat16 *orow = p.out + (((size_t)P.b * p.Nq + i_rel) * p.Hq + h) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tO + c * 32, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
+                                        __uint_as_float(r[2 * e + 1]) * inv_l);
+                if (valid_row) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                }
+            }
+            tc_fence_before();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace swa

@@ -1,0 +1,375 @@
+// swa_api.cu -- host side of libswa: argument checks, TMA descriptors, launch
+// configuration and the device status word.  All kernels are in the headers
+// included below, compiled into this one translation unit.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/swa.h"
+#include "decode_kernel.cuh"
+#include "device_common.cuh"
+#include "prefill_kernel.cuh"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+swa_status_t cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return SWA_ERR_CUDA;
+}
+
+#define SWA_CUDA_TRY(expr)                       \
+    do {                                         \
+        cudaError_t e_ = (expr);                 \
+        if (e_ != cudaSuccess) return cuda_fail(e_); \
+    } while (0)
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ----------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor [d3, d2, d1, d0] (d0 innermost, contiguous) as a 4-D TMA map
+// with a (64, 1, 128, 1) box and 128-byte swizzle: one 128-row x 128-byte
+// region of a K-major UMMA operand per load.  Out-of-range rows read as zero.
+swa_status_t make_operand_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint64_t d3) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};   // bytes, dims 1..3
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = static_cast<int>(r);
+        return SWA_ERR_CUDA;
+    }
+    return SWA_OK;
+}
+
+// ----------------------------------------------------------------- device info
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sms = 0;
+    bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+swa_status_t device_info(DeviceInfo **out) {
+    int dev = 0;
+    SWA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return SWA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.attrs_set) {
+        SWA_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_prefill_kernel<64>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          swa::PrefillCfg<64>::SMEM_ALLOC));
+        SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_prefill_kernel<128>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          swa::PrefillCfg<128>::SMEM_ALLOC));
+#define SWA_SET_DECODE_ATTR(DD, GG)                                                           \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG>,                        \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                      swa::DecodeCfg<DD, GG>::SMEM_BYTES));
+        SWA_SET_DECODE_ATTR(64, 1) SWA_SET_DECODE_ATTR(64, 2) SWA_SET_DECODE_ATTR(64, 4)
+        SWA_SET_DECODE_ATTR(64, 8) SWA_SET_DECODE_ATTR(128, 1) SWA_SET_DECODE_ATTR(128, 2)
+        SWA_SET_DECODE_ATTR(128, 4) SWA_SET_DECODE_ATTR(128, 8)
+#undef SWA_SET_DECODE_ATTR
+        d.attrs_set = true;
+    }
+    *out = &d;
+    return SWA_OK;
+}
+
+// ----------------------------------------------------------------- common checks
+swa_status_t check_heads(int Hq, int Hkv, int D) {
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+    return SWA_OK;
+}
+
+bool bad_scale(float s) { return !(std::isfinite(s) && s > 0.f); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+swa_status_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                            const CUtensorMap &mkc, const CUtensorMap &mvc,
+                            const swa::PrefillParams &p, int sms, cudaStream_t s) {
+    const int grid = p.num_units < sms ? p.num_units : sms;
+    swa::swa_prefill_kernel<D><<<grid, swa::PrefillCfg<D>::THREADS, swa::PrefillCfg<D>::SMEM_ALLOC, s>>>(
+        mq, mk, mv, mkc, mvc, p);
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
+}
+
+swa_status_t launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                           const int32_t *pos, int B, int T, int Hkv, int D, int W, int sms,
+                           cudaStream_t s) {
+    const int row_vec = Hkv * D * 2 / 16;
+    const long long total = (long long)B * T * row_vec;
+    long long blocks = (total + 255) / 256;
+    const long long cap = (long long)sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    swa::swa_append_kernel<<<(int)blocks, 256, 0, s>>>(
+        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), pos, B, T, W, row_vec);
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
+}
+
+int decode_nsplit_max(int W) { return (W + swa::kDecodeSplit - 1) / swa::kDecodeSplit; }
+
+template <int D, int G>
+swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, const int32_t *pos,
+                              void *out, int B, int Hkv, int W, float scale, void *ws,
+                              cudaStream_t s) {
+    const int nsm = decode_nsplit_max(W);
+    const size_t o_elems = (size_t)B * Hkv * nsm * G * D;
+    float *ws_o = static_cast<float *>(ws);
+    float2 *ws_ml = ws ? reinterpret_cast<float2 *>(static_cast<char *>(ws) + ((o_elems * 4 + 255) & ~size_t(255)))
+                       : nullptr;
+    dim3 grid(nsm, Hkv, B);
+    swa::swa_decode_kernel<D, G><<<grid, swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
+        static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
+        Hkv, W, nsm, scale * kLog2e);
+    SWA_CUDA_TRY(cudaGetLastError());
+    if (nsm > 1) {
+        swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), 128, 0, s>>>(
+            pos, ws_ml, ws_o, static_cast<__nv_bfloat16 *>(out), Hkv, W, nsm);
+        SWA_CUDA_TRY(cudaGetLastError());
+    }
+    return SWA_OK;
+}
+
+template <int D>
+swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *vc,
+                             const int32_t *pos, void *out, int B, int Hkv, int W, float scale,
+                             void *ws, cudaStream_t s) {
+    switch (G) {
+        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
+        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
+        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
+        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
+        default: return SWA_ERR_UNSUPPORTED;
+    }
+}
+
+__global__ void swa_selftest_wait_kernel() {
+    __shared__ alignas(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        swa::mbar_init(swa::smem_addr(&bar), 1);
+        abort_flag = 0;
+        swa::mbar_init_fence();
+    }
+    __syncthreads();
+    // nothing ever arrives on `bar`: the wait must run out and record the status
+    swa::mbar_wait_bounded(swa::smem_addr(&bar), 0, &abort_flag, swa::g_wait_limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+swa_status_t swa_prefill(const void *q, const void *k, const void *v, void *out, int B, int N,
+                         int Hq, int Hkv, int D, int W, int window_mode, float scale,
+                         swa_stream_t stream) {
+    if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
+    if (window_mode != SWA_WINDOW_EXCL_LEFT && window_mode != SWA_WINDOW_INCL_LEFT)
+        return SWA_ERR_INVALID_ARG;
+    if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
+    long long Weff = (long long)W + (window_mode == SWA_WINDOW_INCL_LEFT ? 1 : 0);
+    if (Weff > N) Weff = N;                       // the window never reaches before position 0
+    const int G = Hq / Hkv;
+    const long long nqb = (N + 127) / 128;
+    const long long units = (long long)B * Hkv * ((G + 1) / 2) * nqb;
+    if (units > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+
+    CUtensorMap mq, mk, mv;
+    if (swa_status_t e = make_operand_map(&mq, q, D, Hq, N, B)) return e;
+    if (swa_status_t e = make_operand_map(&mk, k, D, Hkv, N, B)) return e;
+    if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, N, B)) return e;
+
+    swa::PrefillParams p{};
+    p.B = B;
+    p.Nq = N;
+    p.Nk = N;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = G;
+    p.W = (int)Weff;
+    p.npairs = (G + 1) / 2;
+    p.nqb = (int)nqb;
+    p.num_units = (int)units;
+    p.scale_log2 = scale * kLog2e;
+    p.chunk_mode = 0;
+    p.start_pos = nullptr;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return D == 128 ? launch_prefill<128>(mq, mk, mv, mk, mv, p, dev->sms, s)
+                    : launch_prefill<64>(mq, mk, mv, mk, mv, p, dev->sms, s);
+}
+
+swa_status_t swa_prefill_chunk(const void *q, const void *k, const void *v, void *k_cache,
+                               void *v_cache, const int32_t *start_pos, void *out, int B, int C,
+                               int Hq, int Hkv, int D, int W, float scale, swa_stream_t stream) {
+    if (!q || !k || !v || !k_cache || !v_cache || !start_pos || !out) return SWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
+        return SWA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || W < 1 || C > W || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
+    if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
+    const int G = Hq / Hkv;
+    const long long nqb = (C + 127) / 128;
+    const long long units = (long long)B * Hkv * ((G + 1) / 2) * nqb;
+    if (units > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+
+    CUtensorMap mq, mk, mv, mkc, mvc;
+    if (swa_status_t e = make_operand_map(&mq, q, D, Hq, C, B)) return e;
+    if (swa_status_t e = make_operand_map(&mk, k, D, Hkv, C, B)) return e;
+    if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, C, B)) return e;
+    if (swa_status_t e = make_operand_map(&mkc, k_cache, D, Hkv, W, B)) return e;
+    if (swa_status_t e = make_operand_map(&mvc, v_cache, D, Hkv, W, B)) return e;
+
+    swa::PrefillParams p{};
+    p.B = B;
+    p.Nq = C;
+    p.Nk = C;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = G;
+    p.W = W;
+    p.npairs = (G + 1) / 2;
+    p.nqb = (int)nqb;
+    p.num_units = (int)units;
+    p.scale_log2 = scale * kLog2e;
+    p.chunk_mode = 1;
+    p.start_pos = start_pos;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    swa_status_t e = D == 128 ? launch_prefill<128>(mq, mk, mv, mkc, mvc, p, dev->sms, s)
+                              : launch_prefill<64>(mq, mk, mv, mkc, mvc, p, dev->sms, s);
+    if (e) return e;
+    // attend first, then write the chunk into the buffer (stream order)
+    return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, s);
+}
+
+swa_status_t swa_cache_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                              const int32_t *pos, int B, int T, int Hkv, int D, int W,
+                              swa_stream_t stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !pos) return SWA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return SWA_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || W < 1 || T > W || Hkv < 1) return SWA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+    return launch_append(k_new, v_new, k_cache, v_cache, pos, B, T, Hkv, D, W, dev->sms,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W) {
+    if (B < 1 || W < 1 || check_heads(Hq, Hkv, D) != SWA_OK) return 0;
+    const size_t nsm = (size_t)decode_nsplit_max(W);
+    const size_t rows = (size_t)B * Hq * nsm;        // (b, kv head, split, head in group)
+    const size_t o_bytes = (rows * D * 4 + 255) & ~size_t(255);
+    return o_bytes + rows * 8;
+}
+
+swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
+                        float scale, void *workspace, size_t workspace_bytes,
+                        swa_stream_t stream) {
+    if (!q || !k_cache || !v_cache || !pos || !out) return SWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return SWA_ERR_INVALID_ARG;
+    if (B < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
+    if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
+    const size_t need = swa_decode_workspace_size(B, Hq, Hkv, D, W);
+    if (decode_nsplit_max(W) > 1) {
+        if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
+    }
+    if (B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+    const int G = Hq / Hkv;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, s)
+                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, s);
+}
+
+swa_status_t swa_get_device_status(swa_stream_t stream) {
+    SWA_CUDA_TRY(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    int v = 0;
+    SWA_CUDA_TRY(cudaMemcpyFromSymbol(&v, swa::g_status, sizeof(int)));
+    const int zero = 0;
+    SWA_CUDA_TRY(cudaMemcpyToSymbol(swa::g_status, &zero, sizeof(int)));
+    return static_cast<swa_status_t>(v);
+}
+
+swa_status_t swa_set_wait_limit_ns(unsigned long long limit_ns) {
+    SWA_CUDA_TRY(cudaMemcpyToSymbol(swa::g_wait_limit_ns, &limit_ns, sizeof(limit_ns)));
+    return SWA_OK;
+}
+
+swa_status_t swa_selftest_wait_timeout(swa_stream_t stream) {
+    swa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
+}
+
+const char *swa_status_string(swa_status_t status) {
+    switch (status) {
+        case SWA_OK: return "SWA_OK";
+        case SWA_ERR_INVALID_ARG: return "SWA_ERR_INVALID_ARG";
+        case SWA_ERR_UNSUPPORTED: return "SWA_ERR_UNSUPPORTED";
+        case SWA_ERR_CUDA: return "SWA_ERR_CUDA";
+        case SWA_ERR_TIMEOUT: return "SWA_ERR_TIMEOUT";
+        default: return "SWA_ERR_UNKNOWN";
+    }
+}
+
+int swa_last_cuda_error(void) { return t_last_cuda_error; }
+
+}  // extern "C"

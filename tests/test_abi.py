@@ -1,0 +1,75 @@
+"""The C ABI library builds for sm_100a, loads without a GPU, exports every
+symbol include/swa.h declares, and rejects bad arguments on the host before
+touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sliding_window_gqa_prefill_b200 as swa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    swa.build()
+    return swa.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "swa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:swa_status_t|size_t|const char \*|int)\s+(swa_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def test_header_declares_the_four_operations():
+    names = declared_symbols()
+    for n in ("swa_prefill", "swa_prefill_chunk", "swa_cache_append", "swa_decode"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", swa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(swa_\w+)$", out, re.M))
+    missing = [n for n in declared_symbols() if n not in exported]
+    assert not missing, missing
+    for n in declared_symbols():
+        assert hasattr(lib, n)
+
+
+def test_null_and_bad_sizes_rejected_without_device(lib):
+    null = None
+    ok_ptr = 0x1000            # aligned, never dereferenced: checks fail first
+    S = swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_prefill(null, ok_ptr, ok_ptr, ok_ptr, 1, 16, 4, 2, 128, 8, 0, 0.1, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr + 2, 1, 16, 4, 2, 128, 8, 0, 0.1, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr, 0, 16, 4, 2, 128, 8, 0, 0.1, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 16, 4, 2, 128, 0, 0, 0.1, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 16, 4, 2, 128, 8, 7, 0.1, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 16, 4, 2, 128, 8, 0, -1.0, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 16, 3, 2, 128, 8, 0, 0.1, None) == S
+    assert lib.swa_prefill(ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 16, 4, 2, 80, 8, 0, 0.1, None) == \
+        swa.SWA_ERR_UNSUPPORTED
+    # chunk longer than the window
+    assert lib.swa_prefill_chunk(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                                 1, 65, 4, 2, 128, 64, 0.1, None) == S
+    # append: T > W, null pos
+    assert lib.swa_cache_append(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 65, 2, 128, 64, None) == S
+    assert lib.swa_cache_append(ok_ptr, ok_ptr, ok_ptr, ok_ptr, null, 1, 1, 2, 128, 64, None) == S
+    # decode: workspace too small
+    assert lib.swa_decode(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, 2, 8, 2, 128, 4096, 0.1,
+                          ok_ptr, 16, None) == S
+
+
+def test_workspace_size_and_status_strings(lib):
+    assert lib.swa_decode_workspace_size(0, 32, 8, 128, 4096) == 0
+    n = lib.swa_decode_workspace_size(64, 32, 8, 128, 4096)
+    # (B*Hq*splits) rows of D floats, then one (m, l) pair per row
+    rows = 64 * 32 * 8
+    assert n == ((rows * 128 * 4 + 255) // 256) * 256 + rows * 8
+    assert lib.swa_status_string(0) == b"SWA_OK"
+    assert lib.swa_status_string(4) == b"SWA_ERR_TIMEOUT"

@@ -1,0 +1,351 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Bar (from the method's accuracy target): bf16 outputs within max-abs 2e-2 and
+mean-abs 2e-3 of the fp64 oracle run on the same bf16 inputs; rolling-buffer
+cache contents bit-exact.  Small cases compare every element; the full-size
+workloads compare sampled rows chosen to hit tile and window edges.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import sliding_window_gqa_prefill_b200 as swa
+from sliding_window_gqa_prefill_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    swa.build()
+    swa.lib()
+    yield
+    assert swa.swa_get_device_status() == swa.SWA_OK
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(gpu: torch.Tensor, ref: np.ndarray, what: str):
+    got = f64(gpu)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    assert err.max() <= MAX_ABS, f"{what}: max-abs {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"{what}: mean-abs {err.mean():.3e}"
+
+
+def run_prefill(q, k, v, W, scale, mode=0):
+    out = swa.swa_prefill(q.cuda(), k.cuda(), v.cuda(), W, scale, window_mode=mode)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+# ------------------------------------------------------------------ one-shot prefill
+
+def test_tiny_workload_full(oracle_mod):
+    """B=1, N=256, W=64, 4 query / 2 KV heads, D=64; fp32 draws rounded to bf16."""
+    w = wl.TINY
+    q, k, v = (t.to(torch.bfloat16) for t in wl.prefill_inputs(w))
+    out = run_prefill(q, k, v, w.W, w.scale)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), w.W, w.scale)
+    assert_close(out, ref, "tiny")
+    # information only: distance to the oracle on the unrounded fp32 draws
+    q32, k32, v32 = wl.prefill_inputs(w)
+    ref32 = oracle_mod.swa_prefill(q32.numpy(), k32.numpy(), v32.numpy(), w.W, w.scale)
+    print(f"tiny: max |gpu - oracle(fp32 inputs)| = {np.abs(f64(out) - ref32).max():.3e}")
+
+
+CASES = [
+    # B, N, Hq, Hkv, D, W
+    (1, 128, 2, 1, 128, 128),      # one tile, dense
+    (1, 300, 4, 2, 128, 64),       # ragged N, W < tile
+    (2, 517, 8, 2, 128, 200),      # W not a multiple of 128, ragged tail, B=2
+    (1, 640, 4, 4, 64, 1),         # W=1: output is v itself (MHA, D=64)
+    (1, 384, 6, 2, 64, 3),         # group of 3 (odd: half-empty head pair)
+    (1, 450, 8, 1, 128, 1000),     # W > N: dense causal, group 8
+    (2, 1024, 8, 2, 128, 256),     # several full bands
+    (1, 257, 2, 2, 64, 129),       # G=1, window one past a tile
+]
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,D,W", CASES)
+def test_prefill_edge_cases(oracle_mod, B, N, Hq, Hkv, D, W):
+    seed = 7 * N + W
+    q = wl.random_bf16((B, N, Hq, D), seed)
+    k = wl.random_bf16((B, N, Hkv, D), seed + 1)
+    v = wl.random_bf16((B, N, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    out = run_prefill(q, k, v, W, scale)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale)
+    assert_close(out, ref, f"prefill B{B} N{N} H{Hq}/{Hkv} D{D} W{W}")
+
+
+def test_prefill_inclusive_window_reading(oracle_mod):
+    B, N, Hq, Hkv, D, W = 1, 400, 4, 2, 128, 100
+    q = wl.random_bf16((B, N, Hq, D), 11)
+    k = wl.random_bf16((B, N, Hkv, D), 12)
+    v = wl.random_bf16((B, N, Hkv, D), 13)
+    out = run_prefill(q, k, v, W, 0.1, mode=swa.SWA_WINDOW_INCL_LEFT)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, 0.1, mode=oracle_mod.WINDOW_INCL_LEFT)
+    assert_close(out, ref, "inclusive window")
+
+
+def test_prefill_large_logits_stable(oracle_mod):
+    """Outlier keys (x8) and a large scale: the lazy-rescaled online softmax
+    must stay finite and accurate."""
+    B, N, Hq, Hkv, D, W = 1, 700, 4, 1, 128, 256
+    q = wl.random_bf16((B, N, Hq, D), 21)
+    k = wl.random_bf16((B, N, Hkv, D), 22)
+    k[:, ::37] *= 8
+    v = wl.random_bf16((B, N, Hkv, D), 23)
+    out = run_prefill(q, k, v, W, 0.3)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, 0.3)
+    assert_close(out, ref, "large logits")
+
+
+def _sample_rows(N, W, extra=48, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = {0, 1, 127, 128, N - 1, N - 128, W - 1, W, W + 1, 2 * W - 1}
+    rows |= set(int(x) for x in rng.integers(0, N, extra))
+    return sorted(r for r in rows if 0 <= r < N)
+
+
+def test_mistral_8k_prefill_sampled(oracle_mod):
+    """B=1, N=8192, W=4096, 32/8 heads, D=128; sampled rows, all heads."""
+    w = wl.MISTRAL_PREFILL_8K
+    q, k, v = wl.prefill_inputs(w)
+    out = run_prefill(q, k, v, w.W, w.scale)
+    rows = _sample_rows(w.N, w.W)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), w.W, w.scale, rows=rows)
+    assert_close(out[:, rows], ref, "mistral 8k (sampled rows)")
+
+
+@pytest.mark.parametrize("N,W", [(16384, 4096), (32768, 4096), (8192, 1024), (4096, 4096)])
+def test_sweep_prefill_sampled(oracle_mod, N, W):
+    """B=2 sweep points with 1% of key rows scaled x8; launch as benchmarked."""
+    w = wl.sweep_point(N, W)
+    q, k, v = wl.prefill_inputs(w)
+    out = run_prefill(q, k, v, w.W, w.scale)
+    rows = _sample_rows(N, W, extra=24, seed=N + W)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), w.W, w.scale, rows=rows)
+    assert_close(out[:, rows], ref, f"sweep N{N} W{W}")
+
+
+def test_dense_control_equals_wide_window():
+    """W >= N (dense causal control) gives the same bits for any W >= N."""
+    B, N, Hq, Hkv, D = 2, 700, 8, 2, 128
+    q = wl.random_bf16((B, N, Hq, D), 31)
+    k = wl.random_bf16((B, N, Hkv, D), 32)
+    v = wl.random_bf16((B, N, Hkv, D), 33)
+    a = run_prefill(q, k, v, N, 0.09)
+    b = run_prefill(q, k, v, 10 * N, 0.09)
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ rolling buffer append
+
+@pytest.mark.parametrize("B,T,Hkv,D,W", [(3, 1, 8, 128, 64), (2, 37, 2, 64, 50), (1, 64, 4, 128, 64),
+                                         (4, 5, 8, 128, 4096)])
+def test_cache_append_bit_exact(oracle_mod, B, T, Hkv, D, W):
+    kc = wl.random_bf16((B, W, Hkv, D), 41)
+    vc = wl.random_bf16((B, W, Hkv, D), 42)
+    kn = wl.random_bf16((B, T, Hkv, D), 43)
+    vn = wl.random_bf16((B, T, Hkv, D), 44)
+    pos = wl.random_positions(B, 0, 3 * W, 45)
+    kg, vg = kc.cuda(), vc.cuda()
+    swa.swa_cache_append(kn.cuda(), vn.cuda(), kg, vg, pos.cuda())
+    torch.cuda.synchronize()
+    kr = kc.view(torch.int16).numpy().copy()
+    vr = vc.view(torch.int16).numpy().copy()
+    oracle_mod.cache_append(kr, vr, None, kn.view(torch.int16).numpy(), vn.view(torch.int16).numpy(), pos.numpy())
+    assert np.array_equal(kg.cpu().view(torch.int16).numpy(), kr)
+    assert np.array_equal(vg.cpu().view(torch.int16).numpy(), vr)
+
+
+# ------------------------------------------------------------------ chunked prefill
+
+def _chunked_case(oracle_mod, B, N, C, Hq, Hkv, D, W, seed, start=0):
+    q = wl.random_bf16((B, N, Hq, D), seed)
+    k = wl.random_bf16((B, N, Hkv, D), seed + 1)
+    v = wl.random_bf16((B, N, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    outs = []
+    for s0 in range(start, N, C):
+        e = min(N, s0 + C)
+        st = torch.full((B,), s0, dtype=torch.int32, device="cuda")
+        outs.append(swa.swa_prefill_chunk(q[:, s0:e].cuda().contiguous(), k[:, s0:e].cuda().contiguous(),
+                                          v[:, s0:e].cuda().contiguous(), kc, vc, st, W, scale))
+    torch.cuda.synchronize()
+    return q, k, v, scale, torch.cat([o.cpu() for o in outs], dim=1), kc.cpu(), vc.cpu()
+
+
+@pytest.mark.parametrize("B,N,C,Hq,Hkv,D,W", [
+    (1, 512, 128, 4, 2, 128, 128),    # C = W aligned
+    (2, 700, 96, 4, 2, 128, 256),     # C < W, unaligned starts
+    (1, 600, 200, 8, 2, 64, 200),     # W not a multiple of 128, C = W
+    (1, 333, 45, 2, 1, 128, 100),     # small ragged chunks
+    (1, 1100, 300, 6, 2, 128, 384),   # odd group, wrap inside tiles
+])
+def test_chunked_prefill_matches_oracle(oracle_mod, B, N, C, Hq, Hkv, D, W):
+    q, k, v, scale, out, kc, vc = _chunked_case(oracle_mod, B, N, C, Hq, Hkv, D, W, seed=N + C)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale)
+    assert_close(out, ref, f"chunked N{N} C{C} W{W}")
+    # cache: slot s holds the last position p < N with p mod W == s, bit for bit
+    for s in range(min(W, N)):
+        p = s + ((N - 1 - s) // W) * W
+        assert torch.equal(kc[:, s], k[:, p]) and torch.equal(vc[:, s], v[:, p]), (s, p)
+
+
+def test_chunked_16k_workload(oracle_mod):
+    """N=16384 in 4 chunks of 4096 through a W=4096 buffer, 32/8 heads, D=128:
+    sampled rows vs one-shot oracle; final cache = positions 12288..16383."""
+    w = wl.CHUNKED_16K
+    q, k, v = wl.chunked_inputs(w)
+    kc = torch.zeros(w.B, w.W, w.Hkv, w.D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    outs = []
+    for s0 in range(0, w.N, w.C):
+        st = torch.full((w.B,), s0, dtype=torch.int32, device="cuda")
+        outs.append(swa.swa_prefill_chunk(qg[:, s0:s0 + w.C].contiguous(), kg[:, s0:s0 + w.C].contiguous(),
+                                          vg[:, s0:s0 + w.C].contiguous(), kc, vc, st, w.W, w.scale))
+    out = torch.cat(outs, dim=1).cpu()
+    rows = _sample_rows(w.N, w.W, extra=40, seed=3)
+    rows += [w.C - 1, w.C, 2 * w.C - 1, 2 * w.C, 3 * w.C + 5]
+    rows = sorted(set(rows))
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), w.W, w.scale, rows=rows)
+    assert_close(out[:, rows], ref, "chunked 16k (sampled rows)")
+    assert torch.equal(kc.cpu(), k[:, w.N - w.W:]) and torch.equal(vc.cpu(), v[:, w.N - w.W:])
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps, seed):
+    kc = wl.random_bf16((B, W, Hkv, D), seed)
+    vc = wl.random_bf16((B, W, Hkv, D), seed + 1)
+    qs = wl.random_bf16((steps, B, Hq, D), seed + 2)
+    kn = wl.random_bf16((steps, B, Hkv, D), seed + 3)
+    vn = wl.random_bf16((steps, B, Hkv, D), seed + 4)
+    scale = 1.0 / math.sqrt(D)
+    kg, vg = kc.cuda(), vc.cuda()
+    pos0 = torch.as_tensor(pos0, dtype=torch.int32)
+    sp = oracle_mod.slot_positions(pos0.numpy(), W)
+    kr, vr = f64(kc), f64(vc)
+    for s in range(steps):
+        pos = (pos0 + s).to(torch.int32)
+        pg = pos.cuda()
+        swa.swa_cache_append(kn[s].unsqueeze(1).cuda(), vn[s].unsqueeze(1).cuda(), kg, vg, pg)
+        out = swa.swa_decode(qs[s].cuda(), kg, vg, pg, scale)
+        torch.cuda.synchronize()
+        oracle_mod.cache_append(kr, vr, sp, f64(kn[s].unsqueeze(1)), f64(vn[s].unsqueeze(1)), pos.numpy())
+        ref = oracle_mod.swa_decode(f64(qs[s]), kr, vr, sp, pos.numpy(), W, scale)
+        assert_close(out.cpu(), ref, f"decode step {s}")
+    assert np.array_equal(f64(kg.cpu()), kr) and np.array_equal(f64(vg.cpu()), vr)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,W,pos0", [
+    (4, 32, 8, 128, 4096, [0, 1, 4094, 4095]),          # partial buffer, last slot, first wrap
+    (3, 8, 2, 128, 4096, [4096, 8191, 30000]),          # wrap points and deep positions
+    (2, 4, 4, 64, 700, [10, 2000]),                     # G=1, W not a multiple of 512
+    (2, 16, 2, 128, 1000, [999, 5]),                    # G=8
+    (2, 4, 2, 64, 300, [299, 77]),                      # G=2, single split
+])
+def test_decode_edge_cases(oracle_mod, B, Hq, Hkv, D, W, pos0):
+    _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps=3, seed=B * W + D)
+
+
+def test_decode_b64_workload(oracle_mod):
+    """B=64, W=4096, 32/8 heads, D=128, positions uniform on [1, 32768]: first
+    three of the 128 steps against the oracle, cache bit-exact."""
+    w = wl.DECODE_B64
+    d = wl.decode_inputs(w)
+    kg, vg = d["k_cache"].cuda(), d["v_cache"].cuda()
+    sp = oracle_mod.slot_positions(d["pos0"].numpy(), w.W)
+    kr, vr = f64(d["k_cache"]), f64(d["v_cache"])
+    for s in range(3):
+        pos = (d["pos0"] + s).to(torch.int32)
+        pg = pos.cuda()
+        swa.swa_cache_append(d["k_new"][s].unsqueeze(1).cuda(), d["v_new"][s].unsqueeze(1).cuda(), kg, vg, pg)
+        out = swa.swa_decode(d["q"][s].cuda(), kg, vg, pg, w.scale)
+        torch.cuda.synchronize()
+        oracle_mod.cache_append(kr, vr, sp, f64(d["k_new"][s].unsqueeze(1)), f64(d["v_new"][s].unsqueeze(1)),
+                                pos.numpy())
+        ref = oracle_mod.swa_decode(f64(d["q"][s]), kr, vr, sp, pos.numpy(), w.W, w.scale)
+        assert_close(out.cpu(), ref, f"decode B64 step {s}")
+    assert np.array_equal(f64(kg.cpu()), kr) and np.array_equal(f64(vg.cpu()), vr)
+
+
+def test_prefill_then_decode_continues_the_sequence(oracle_mod):
+    """Chunked prefill leaves the buffer in the state decode continues from:
+    decode at position N equals row N of one-shot SWA over N+1 tokens."""
+    B, N, C, Hq, Hkv, D, W = 1, 600, 256, 8, 2, 128, 256
+    q = wl.random_bf16((B, N + 1, Hq, D), 51)
+    k = wl.random_bf16((B, N + 1, Hkv, D), 52)
+    v = wl.random_bf16((B, N + 1, Hkv, D), 53)
+    scale = 1.0 / math.sqrt(D)
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    for s0 in range(0, N, C):
+        e = min(N, s0 + C)
+        st = torch.full((B,), s0, dtype=torch.int32, device="cuda")
+        swa.swa_prefill_chunk(q[:, s0:e].cuda().contiguous(), k[:, s0:e].cuda().contiguous(),
+                              v[:, s0:e].cuda().contiguous(), kc, vc, st, W, scale)
+    pos = torch.full((B,), N, dtype=torch.int32, device="cuda")
+    swa.swa_cache_append(k[:, N:].cuda().contiguous(), v[:, N:].cuda().contiguous(), kc, vc, pos)
+    out = swa.swa_decode(q[:, N].cuda().contiguous(), kc, vc, pos, scale)
+    ref = oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale, rows=[N])
+    assert_close(out.cpu(), ref[:, 0], "prefill -> decode")
+
+
+# ------------------------------------------------------------------ failure paths (no fault)
+
+def test_timeout_path_reports_status_and_context_survives(oracle_mod):
+    swa.swa_set_wait_limit_ns(2_000_000)            # 2 ms
+    try:
+        swa.swa_selftest_wait_timeout()
+        assert swa.swa_get_device_status() == swa.SWA_ERR_TIMEOUT
+    finally:
+        swa.swa_set_wait_limit_ns(1_000_000_000)
+    assert swa.swa_get_device_status() == swa.SWA_OK
+    test_prefill_edge_cases(oracle_mod, 1, 300, 4, 2, 128, 64)
+
+
+def test_negative_position_is_reported_not_faulted():
+    B, W, Hkv, D = 2, 64, 2, 64
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kn = torch.ones(B, 1, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    pos = torch.tensor([-5, 3], dtype=torch.int32, device="cuda")
+    swa.swa_cache_append(kn, kn, kc, vc, pos)
+    assert swa.swa_get_device_status() == swa.SWA_ERR_INVALID_ARG
+    assert kc[0].abs().sum().item() == 0 and kc[1, 3].abs().sum().item() > 0
+
+
+def test_host_side_validation_errors():
+    q = torch.zeros(1, 16, 4, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 16, 2, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(swa.SwaError) as e:
+        swa.swa_prefill(q, k, k, 0, 0.1)             # W = 0
+    assert e.value.status == swa.SWA_ERR_INVALID_ARG
+    with pytest.raises(swa.SwaError) as e:
+        swa.swa_prefill(q, k, k, 4, float("nan"))
+    assert e.value.status == swa.SWA_ERR_INVALID_ARG
+    q3 = torch.zeros(1, 16, 3, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(swa.SwaError) as e:
+        swa.swa_prefill(q3, k, k, 4, 0.1)            # Hq % Hkv != 0
+    assert e.value.status == swa.SWA_ERR_INVALID_ARG
+    q96 = torch.zeros(1, 16, 4, 96, dtype=torch.bfloat16, device="cuda")
+    k96 = torch.zeros(1, 16, 2, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(swa.SwaError) as e:
+        swa.swa_prefill(q96, k96, k96, 4, 0.1)       # head_dim 96
+    assert e.value.status == swa.SWA_ERR_UNSUPPORTED
