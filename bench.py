@@ -153,14 +153,21 @@ def dist_setup(gpus: int):
     return rank, world, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Maximum of a per-rank scalar (a time) over all ranks."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: every rank processes the same units; the job
+    takes as long as its slowest rank."""
+    return units_per_rank * world / max_seconds
 
 
 def barrier(world: int):
@@ -310,11 +317,11 @@ def run_native(args):
     de_total = max_over_ranks(sum(de_ms), world)
     step_total = max_over_ranks(total_ms, world)
 
-    value = pf_flops * args.steps * world / (pf_total * 1e-3) / 1e12
+    value = weak_scaling_rate(pf_flops * args.steps, world, pf_total * 1e-3) / 1e12
     pf_avg_ms = pf_total / args.steps
     achieved = pf_flops / (pf_avg_ms * 1e-3) / 1e12
-    chunk_tflops = c_flops * args.steps * world / (ch_total * 1e-3) / 1e12
-    dec_tok_s = dw.B * dw.steps * args.steps * world / (de_total * 1e-3)
+    chunk_tflops = weak_scaling_rate(c_flops * args.steps, world, ch_total * 1e-3) / 1e12
+    dec_tok_s = weak_scaling_rate(dw.B * dw.steps * args.steps, world, de_total * 1e-3)
     dec_gbs = (kv_bytes + other_bytes) / ((de_total / args.steps) * 1e-3) / 1e9
     dec_kv_gbs = kv_bytes / ((de_total / args.steps) * 1e-3) / 1e9
 
@@ -341,7 +348,7 @@ def run_native(args):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = pf_flops * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = weak_scaling_rate(pf_flops * args.steps, world, e2e_ms * 1e-3) / 1e12
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = hout.numel() * 2
 
