@@ -137,6 +137,39 @@ swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
 size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W);
 
 /*
+ * swa_decode_noalloc -- swa_decode without a caller-provided workspace.
+ * The pages have no counterpart: this is an interface convenience only.
+ *
+ * Some callers cannot hand the library scratch memory.  A plug-in hosted by
+ * an application that owns all device memory through its own pool may not
+ * call cudaMalloc at all; a latency-critical serving loop cannot afford it,
+ * because cudaMalloc may synchronise the device and stall every stream; and a
+ * caller that plans its memory budget once at start-up has no way to grow it
+ * per request.
+ * This entry point takes the same inputs and outputs as swa_decode but keeps
+ * its split partials in a scratch array that the library reserves statically
+ * in device memory: SWA_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) on every GPU
+ * where the library is loaded, held until the process exits.  It allocates
+ * nothing and calls no allocating routine.
+ *
+ * Limits and behaviour:
+ *  - sizes whose workspace (swa_decode_workspace_size) exceeds
+ *    SWA_DECODE_NOALLOC_SCRATCH_BYTES are rejected with SWA_ERR_UNSUPPORTED
+ *    before anything is launched (B=64, Hq=32, D=128, W=4096 needs 8.5 MB);
+ *  - the first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture;
+ *  - all calls share the one array and it keeps the last call's contents;
+ *    nothing in it needs to start at zero.  Calls that overlap on the GPU
+ *    (different streams, or different host threads without ordering) race on
+ *    it and give wrong results: serialise them.
+ */
+#define SWA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+swa_status_t swa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *pos, void *out, int B, int Hq, int Hkv, int D,
+                                int W, float scale, swa_stream_t stream);
+
+/*
  * swa_get_device_status -- synchronise `stream`, then return (and reset to
  * SWA_OK) the device status word that kernels of this library set when a
  * bounded wait runs out.  Returns SWA_ERR_CUDA if synchronisation fails.

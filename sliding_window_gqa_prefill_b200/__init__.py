@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.swa_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, st]
             L.swa_cache_append.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, st]
             L.swa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, ctypes.c_size_t, st]
+            L.swa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, st]
+            L.swa_decode_noalloc.restype = ctypes.c_int
             L.swa_decode_workspace_size.argtypes = [i, i, i, i, i]
             L.swa_decode_workspace_size.restype = ctypes.c_size_t
             L.swa_get_device_status.argtypes = [st]

@@ -199,6 +199,30 @@ __global__ void swa_selftest_wait_kernel() {
     swa::mbar_wait_bounded(swa::smem_addr(&bar), 0, &abort_flag, swa::g_wait_limit_ns);
 }
 
+// Scratch of swa_decode_noalloc: reserved statically on every device that
+// loads this library, shared by all its calls.  Host code must not pass the
+// symbol itself to a kernel (on the host it names a host-side shadow); the
+// device address is looked up once per device with cudaGetSymbolAddress.
+constexpr size_t kNoallocScratchBytes = SWA_DECODE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+void *g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+swa_status_t noalloc_scratch(void **out) {
+    int dev = 0;
+    SWA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return SWA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        SWA_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));   // device `dev` is current
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SWA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -337,6 +361,27 @@ swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, s)
                     : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, s);
+}
+
+swa_status_t swa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *pos, void *out, int B, int Hq, int Hkv, int D,
+                                int W, float scale, swa_stream_t stream) {
+    if (!q || !k_cache || !v_cache || !pos || !out) return SWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return SWA_ERR_INVALID_ARG;
+    if (B < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
+    if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
+    if (swa_decode_workspace_size(B, Hq, Hkv, D, W) > kNoallocScratchBytes) return SWA_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if (swa_status_t e = noalloc_scratch(&scratch)) return e;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int G = Hq / Hkv;
+    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, scratch, s)
+                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, scratch, s);
 }
 
 swa_status_t swa_get_device_status(swa_stream_t stream) {
