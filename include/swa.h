@@ -192,6 +192,15 @@ swa_status_t swa_set_wait_limit_ns(unsigned long long limit_ns);
  */
 swa_status_t swa_selftest_wait_timeout(swa_stream_t stream);
 
+/*
+ * swa_selftest_exp2 -- test hook: y[i] = 2^x[i] computed by the FMA-pipe
+ * exponential the prefill kernel uses for a share of its softmax
+ * (polynomial after Cody-Waite range reduction; relative error below 2e-4
+ * for x >= -126; inputs below -126, -inf included, give values in
+ * [0, 2^-125]).  x, y: n floats in device memory.
+ */
+swa_status_t swa_selftest_exp2(const float *x, float *y, int n, swa_stream_t stream);
+
 /* Human-readable name of a status code. */
 const char *swa_status_string(swa_status_t status);
 

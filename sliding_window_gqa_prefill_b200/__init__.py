@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
             L.swa_get_device_status.argtypes = [st]
             L.swa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
             L.swa_selftest_wait_timeout.argtypes = [st]
+            L.swa_selftest_exp2.argtypes = [vp, vp, i, st]
+            L.swa_selftest_exp2.restype = ctypes.c_int
             L.swa_status_string.argtypes = [i]
             L.swa_status_string.restype = ctypes.c_char_p
             L.swa_last_cuda_error.argtypes = []
@@ -198,6 +200,17 @@ def swa_get_device_status(stream=None) -> int:
 
 def swa_set_wait_limit_ns(limit_ns: int) -> None:
     _check(lib().swa_set_wait_limit_ns(int(limit_ns)), "swa_set_wait_limit_ns")
+
+
+def swa_selftest_exp2(x, stream=None):
+    """2^x by the prefill kernel's FMA-pipe exponential (test hook); x float32 CUDA."""
+    import torch
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise TypeError("x: expected a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check(lib().swa_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream_handle(stream)),
+           "swa_selftest_exp2")
+    return y
 
 
 def swa_selftest_wait_timeout(stream=None) -> None:

@@ -75,6 +75,9 @@ struct PrefillCfg {
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-byte alignment
     static constexpr int THREADS = 384;
+    // which of the 16 column pairs of each 32-column chunk take the polynomial
+    // exponential instead of ex2.approx (bits 3, 7, 11, 15: one pair in four)
+    static constexpr uint32_t kEmuPairs = 0x8888u;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, 1);
@@ -419,13 +422,17 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 ++sc;
                 tc_fence_after();
                 float s[BN];
+                {
+                    uint32_t r[BN / 32][32];
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + c * 32, r);
+                    for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, r[c]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+                    for (int c = 0; c < BN / 32; ++c) {
+                        reg_fence32(r[c]);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[c][e]);
+                    }
                 }
                 if (T.masked) {
                     if (T.cache) {
@@ -445,9 +452,15 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         }
                     }
                 }
-                float mt = s[0];
+                float mx[8];
 #pragma unroll
-                for (int c = 1; c < BN; ++c) mt = fmaxf(mt, s[c]);
+                for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+                for (int c = 8; c < BN; c += 8)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
+                const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                 const float m_tile = mt * sl2;
                 const float m_cand = fmaxf(m_use, m_tile);
                 if (j == 0) {
@@ -473,20 +486,27 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-                float lsum = 0.f;
+                const float2 sl2x2 = make_float2(sl2, sl2), nmb2 = make_float2(-mb, -mb);
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < BN / 32; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * e], sl2, -mb));
-                        const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * e + 1], sl2, -mb));
-                        lsum += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
+                        const float2 x = ffma2(make_float2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sl2x2, nmb2);
+                        // a share of the exponentials runs on the FMA pipe (kEmuPairs bit e)
+                        const float2 pe = ((Cfg::kEmuPairs >> e) & 1u)
+                                              ? exp2_poly2(x)
+                                              : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        acc[e & 3] = fadd2(acc[e & 3], pe);
+                        pk[e] = pack_bf16x2(pe.x, pe.y);
                     }
                     tmem_st16(tS + c * 16, pk);
                 }
-                l += lsum;
+                const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+                const float2 asum = fadd2(a01, a23);
+                l += asum.x + asum.y;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();

@@ -223,6 +223,17 @@ swa_status_t noalloc_scratch(void **out) {
     return SWA_OK;
 }
 
+__global__ void swa_selftest_exp2_kernel(const float *x, float *y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i + 1 < n) {
+        const float2 r = swa::exp2_poly2(make_float2(x[i], x[i + 1]));
+        y[i] = r.x;
+        y[i + 1] = r.y;
+    } else if (i < n) {
+        y[i] = swa::exp2_poly2(make_float2(x[i], 0.f)).x;
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -400,6 +411,14 @@ swa_status_t swa_set_wait_limit_ns(unsigned long long limit_ns) {
 
 swa_status_t swa_selftest_wait_timeout(swa_stream_t stream) {
     swa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
+}
+
+swa_status_t swa_selftest_exp2(const float *x, float *y, int n, swa_stream_t stream) {
+    if (!x || !y || n < 1) return SWA_ERR_INVALID_ARG;
+    const int pairs = (n + 1) / 2;
+    swa_selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
     SWA_CUDA_TRY(cudaGetLastError());
     return SWA_OK;
 }

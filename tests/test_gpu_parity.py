@@ -307,6 +307,24 @@ def test_prefill_then_decode_continues_the_sequence(oracle_mod):
     assert_close(out.cpu(), ref[:, 0], "prefill -> decode")
 
 
+# ------------------------------------------------------------------ FMA-pipe exponential
+
+def test_polynomial_exp2_against_cuda_exp2():
+    """The softmax's polynomial 2^x against CUDA's exp2f (torch.exp2) on the
+    range it sees (x <= 8 after max subtraction), plus masked inputs."""
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1_000_003, device="cuda"),
+                   torch.rand(1_000_000, device="cuda") * 20 - 12]).contiguous()
+    y = swa.swa_selftest_exp2(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    # fit error 7.5e-5 plus fp32 rounding of coefficients and Horner steps;
+    # P is stored in bf16 (relative step 2^-8), so 2e-4 is far below what matters
+    assert rel < 2e-4, rel
+    lo = torch.tensor([-126.5, -127.0, -200.0, -1e30, float("-inf")], device="cuda")
+    ylo = swa.swa_selftest_exp2(lo)
+    assert bool(((ylo >= 0) & (ylo <= 2.0 ** -125)).all()), ylo.tolist()
+
+
 # ------------------------------------------------------------------ failure paths (no fault)
 
 def test_timeout_path_reports_status_and_context_survives(oracle_mod):
