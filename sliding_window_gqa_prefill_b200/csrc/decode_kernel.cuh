@@ -63,6 +63,27 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// G consecutive floats of shared memory, vectorised where G allows.
+template <int G>
+__device__ __forceinline__ void load_g(const float *p, float (&out)[G]) {
+    if constexpr (G % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < G / 4; ++i) {
+            const float4 t = reinterpret_cast<const float4 *>(p)[i];
+            out[4 * i] = t.x;
+            out[4 * i + 1] = t.y;
+            out[4 * i + 2] = t.z;
+            out[4 * i + 3] = t.w;
+        }
+    } else if constexpr (G == 2) {
+        const float2 t = *reinterpret_cast<const float2 *>(p);
+        out[0] = t.x;
+        out[1] = t.y;
+    } else {
+        out[0] = p[0];
+    }
+}
+
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -105,14 +126,16 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const uint32_t ring = smem_addr(smem + warp * Cfg::WARP_RING);
     float *score = reinterpret_cast<float *>(smem + Cfg::OFF_SCORE) + warp * KI * G;
 
-    // q for every head of the group, d = sub*8 .. sub*8+7, pre-scaled to base 2
-    float qf[G][8];
+    // q for every head of the group, d = sub*8 .. sub*8+7, pre-scaled to base 2,
+    // as four (even, odd) pairs for the packed two-lane FMA
+    float2 q2[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)b * Hq + g * G + h) * D) + sub);
-        bf16x8_to_f32(raw, qf[h]);
+        float qf[8];
+        bf16x8_to_f32(raw, qf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qf[h][e] *= scale_log2;
+        for (int e = 0; e < 4; ++e) q2[h][e] = make_float2(qf[2 * e] * scale_log2, qf[2 * e + 1] * scale_log2);
     }
 
     const size_t row_stride = (size_t)Hkv * D;     // elements between consecutive slots
@@ -136,13 +159,18 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         }
     };
 
-    float m_run[G], l_run[G], o[G][8];
+    // m_run: running base-2 maximum per head (equal in all lanes);
+    // l_run: this lane's share of the running sum per head (each key x head
+    // is counted by exactly one lane); o2: this lane's row-group partial of
+    // the output for its 8 d, per head
+    float m_run[G], l_run[G];
+    float2 o2[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         m_run[h] = -INFINITY;
         l_run[h] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[h][e] = 0.f;
+        for (int e = 0; e < 4; ++e) o2[h][e] = make_float2(0.f, 0.f);
     }
 
 #pragma unroll
@@ -151,7 +179,8 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         cp_async_commit();
     }
 
-    // value index of v[i] after the butterfly = vbase_idx + i
+    // value index of v[i] after the butterfly = vidx0 + i; lanes that only
+    // hold copies (when NV < LPR) do not write
     int vidx0 = 0;
     {
         int half = NV;
@@ -162,6 +191,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             if (sub & off) vidx0 += half;
         }
     }
+    const bool writer = (TLEV == ilog2c(LPR)) || ((sub & ((LPR >> TLEV) - 1)) == 0);
 
     for (int it_local = 0; it_local < my_iters; ++it_local) {
         const int stage = it_local % kDecodeStages;
@@ -176,7 +206,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         const int it = warp + it_local * kDecodeWarps;
         const int key_base = begin + it * KI;
 
-        // partial dot products: value index kk*G + h
+        // partial dot products over this lane's 8 d: value index kk*G + h
         float v[NV];
 #pragma unroll
         for (int kk = 0; kk < KPR; ++kk) {
@@ -185,91 +215,126 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             bf16x8_to_f32(*reinterpret_cast<const uint4 *>(st + (kr * D + sub * 8) * 2), kf);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                float acc = 0.f;
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc = fmaf(qf[h][e], kf[e], acc);
-                v[kk * G + h] = acc;
+                for (int e = 0; e < 4; ++e) acc = ffma2(q2[h][e], make_float2(kf[2 * e], kf[2 * e + 1]), acc);
+                v[kk * G + h] = acc.x + acc.y;
             }
         }
         // transposing butterfly across the LPR lanes of the row
-        {
 #pragma unroll
-            for (int lev = 0; lev < ilog2c(LPR); ++lev) {
-                const int off = LPR >> (lev + 1);
-                if (lev < TLEV) {
-                    const int half = NV >> (lev + 1);
-                    const bool upper = (sub & off) != 0;
+        for (int lev = 0; lev < ilog2c(LPR); ++lev) {
+            const int off = LPR >> (lev + 1);
+            if (lev < TLEV) {
+                const int half = NV >> (lev + 1);
+                const bool upper = (sub & off) != 0;
 #pragma unroll
-                    for (int i = 0; i < NV / 2; ++i) {
-                        if (i < half) {
-                            const float send = upper ? v[i] : v[i + half];
-                            const float keep = upper ? v[i + half] : v[i];
-                            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                        }
+                for (int i = 0; i < NV / 2; ++i) {
+                    if (i < half) {
+                        const float send = upper ? v[i] : v[i + half];
+                        const float keep = upper ? v[i + half] : v[i];
+                        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < VPL; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
                 }
+            } else {
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
             }
         }
-        // scores to shared memory (one writer per value), masking keys past the split
-        if (TLEV == ilog2c(LPR) || (sub & ((LPR >> TLEV) - 1)) == 0) {
+        // scores of this iteration to shared memory, [KI][G]; keys past the split masked
+        if (writer) {
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
                 const int idx = vidx0 + i;
-                const int kk = idx / G, h = idx % G;
-                const int kr = row * KPR + kk;
-                score[kr * G + h] = (key_base + kr < end) ? v[i] : -INFINITY;
+                const int kr = row * KPR + idx / G;
+                v[i] = (key_base + kr < end) ? v[i] : -INFINITY;
+                score[kr * G + idx % G] = v[i];
             }
         }
         __syncwarp();
-        // iteration maximum per head, then lazy-free exact online update
         float m_new[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) m_new[h] = m_run[h];
 #pragma unroll
-        for (int kr = 0; kr < KI; ++kr)
+        for (int kr = 0; kr < KI; ++kr) {
+            float sv[G];
+            load_g<G>(score + kr * G, sv);
 #pragma unroll
-            for (int h = 0; h < G; ++h) m_new[h] = fmaxf(m_new[h], score[kr * G + h]);
+            for (int h = 0; h < G; ++h) m_new[h] = fmaxf(m_new[h], sv[h]);
+        }
+        __syncwarp();                        // every lane has read the scores
+        bool grow = false;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            if (m_new[h] > m_run[h]) {
-                const float alpha = ex2_approx(m_run[h] - m_new[h]);
+        for (int h = 0; h < G; ++h) grow |= m_new[h] > m_run[h];
+        if (grow) {                          // uniform across the warp
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float alpha = ex2_approx(m_run[h] - m_new[h]);   // 0 when m_run = -inf
                 l_run[h] *= alpha;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[h][e] *= alpha;
+                for (int e = 0; e < 4; ++e) o2[h][e] = make_float2(o2[h][e].x * alpha, o2[h][e].y * alpha);
                 m_run[h] = m_new[h];
             }
         }
+        // one exponential per key x head, by the lane that holds it
+        if (writer) {
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int idx = vidx0 + i;
+                const int kr = row * KPR + idx / G, h = idx % G;
+                float mh = m_run[0];
+#pragma unroll
+                for (int hh = 1; hh < G; ++hh) mh = (h == hh) ? m_run[hh] : mh;
+                const float pw = ex2_approx(v[i] - mh);
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh) l_run[hh] += (h == hh) ? pw : 0.f;
+                score[kr * G + h] = pw;
+            }
+        }
+        __syncwarp();
         // P V for the KPR keys of this lane's row
 #pragma unroll
         for (int kk = 0; kk < KPR; ++kk) {
             const int kr = row * KPR + kk;
             float vf[8];
             bf16x8_to_f32(*reinterpret_cast<const uint4 *>(st + KI * D * 2 + (kr * D + sub * 8) * 2), vf);
+            float pw[G];
+            load_g<G>(score + kr * G, pw);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                const float pw = ex2_approx(score[kr * G + h] - m_run[h]);
-                l_run[h] += pw;
+                const float2 p2 = make_float2(pw[h], pw[h]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pw, vf[e], o[h][e]);
+                for (int e = 0; e < 4; ++e) o2[h][e] = ffma2(p2, make_float2(vf[2 * e], vf[2 * e + 1]), o2[h][e]);
             }
         }
         __syncwarp();
     }
     cp_async_wait<0>();
 
-    // merge the row groups of the warp (lanes with equal sub)
+    // merge within the warp: o over the row groups (lanes with equal sub),
+    // l over every lane
 #pragma unroll
     for (int off = LPR; off < 32; off <<= 1) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], off);
+        for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], off);
-        }
+            for (int e = 0; e < 4; ++e) {
+                o2[h][e].x += __shfl_xor_sync(0xffffffffu, o2[h][e].x, off);
+                o2[h][e].y += __shfl_xor_sync(0xffffffffu, o2[h][e].y, off);
+            }
     }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < G; ++h) l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], off);
+    float o[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            o[h][2 * e] = o2[h][e].x;
+            o[h][2 * e + 1] = o2[h][e].y;
+        }
     // merge the warps of the block in shared memory
     float *mg = reinterpret_cast<float *>(smem + Cfg::OFF_MERGE);    // [warp][G][D+2]
     if (row == 0) {
@@ -322,16 +387,41 @@ swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restr
     const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
     if (nsplit <= 1) return;
     const size_t base = (size_t)(b * Hkv + g) * nsplit_max;
+    constexpr int kUnrolled = 16;            // splits loaded side by side (W <= 8192)
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D, d = idx % D;
-        float m = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) m = fmaxf(m, ws_ml[(base + s) * G + h].x);
-        float l = 0.f, acc = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const float2 ml = ws_ml[(base + s) * G + h];
-            const float sc = ex2_approx(ml.x - m);
-            l += ml.y * sc;
-            acc += ws_o[((base + s) * G + h) * D + d] * sc;
+        float m = -INFINITY, l = 0.f, acc = 0.f;
+        if (nsplit <= kUnrolled) {
+            float ms[kUnrolled], ls[kUnrolled], os[kUnrolled];
+#pragma unroll
+            for (int s = 0; s < kUnrolled; ++s) {
+                if (s < nsplit) {
+                    const float2 ml = ws_ml[(base + s) * G + h];
+                    ms[s] = ml.x;
+                    ls[s] = ml.y;
+                    os[s] = ws_o[((base + s) * G + h) * D + d];
+                } else {
+                    ms[s] = -INFINITY;
+                    ls[s] = 0.f;
+                    os[s] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int s = 0; s < kUnrolled; ++s) m = fmaxf(m, ms[s]);
+#pragma unroll
+            for (int s = 0; s < kUnrolled; ++s) {
+                const float sc = (s < nsplit) ? ex2_approx(ms[s] - m) : 0.f;
+                l += ls[s] * sc;
+                acc += os[s] * sc;
+            }
+        } else {
+            for (int s = 0; s < nsplit; ++s) m = fmaxf(m, ws_ml[(base + s) * G + h].x);
+            for (int s = 0; s < nsplit; ++s) {
+                const float2 ml = ws_ml[(base + s) * G + h];
+                const float sc = ex2_approx(ml.x - m);
+                l += ml.y * sc;
+                acc += ws_o[((base + s) * G + h) * D + d] * sc;
+            }
         }
         out[((size_t)b * Hq + g * G + h) * D + d] = __float2bfloat16_rn(acc / l);
     }

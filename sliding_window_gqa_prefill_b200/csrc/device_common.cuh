@@ -64,17 +64,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of the same condition (no suspension of the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase of parity `parity` of barrier `bar` has completed.
 // Bounded: gives up when *abort becomes non-zero (another thread of the block
 // gave up) or after `limit_ns`; on running out it records SWA_ERR_TIMEOUT,
 // raises *abort and returns false.  Never traps.
+// kSpin: poll without suspending (for a latency-critical single thread).
+template <bool kSpin = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int *abort,
                                                   unsigned long long limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t spin = 1;; ++spin) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if ((spin & 31u) == 0u) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 >= limit_ns) {
@@ -249,6 +264,21 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
     return d;
 }
 
+// The same descriptor as two 32-bit words.  lo holds the start address and
+// the leading byte offset, hi the stride byte offset, version and swizzle, so
+// stepping a descriptor along K inside a 128-byte swizzle row, or from one
+// tile slot to the next, is a single 32-bit add on lo (the 14-bit address
+// field of shared memory below 256 KB never carries into the offset field).
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((uint32_t)kSwizzle128B << 29);
+}
+__device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t smem_desc64(uint32_t lo, uint32_t hi) {
+    return ((uint64_t)hi << 32) | lo;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, bf16 A
 // and B, A K-major, B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int b_mn_major) {
@@ -313,6 +343,12 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     p = ffma2(p, f, make_float2(c0, c0));
     return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
                        __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

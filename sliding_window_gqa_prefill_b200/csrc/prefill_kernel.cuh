@@ -69,8 +69,8 @@ struct PrefillCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST],
-    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain
-    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1;
+    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain, p_half[2]
+    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-byte alignment
@@ -78,6 +78,13 @@ struct PrefillCfg {
     // which of the 16 column pairs of each 32-column chunk take the polynomial
     // exponential instead of ex2.approx (bits 3, 7, 11, 15: one pair in four)
     static constexpr uint32_t kEmuPairs = 0x8888u;
+    // PV in two halves of 64 keys: the first half starts while the softmax
+    // still computes the second half of P
+    static constexpr bool kSplitPV = true;
+    // row maximum with three-input max instructions
+    static constexpr bool kMax3 = false;
+    // the MMA thread polls its barriers instead of suspending on them
+    static constexpr bool kMmaSpin = false;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, 1);
@@ -215,6 +222,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t bar_p_full = bar_s_full + 16;
     const uint32_t bar_o_full = bar_p_full + 16;
     const uint32_t bar_drain = bar_o_full + 16;
+    const uint32_t bar_p_half = bar_drain + 8;                // + 8*t
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::OFF_MISC + 4);
 
@@ -239,6 +247,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_init(bar_o_full + 8 * t, 1);
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_p_half, 4);
+        mbar_init(bar_p_half + 8, 4);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -311,36 +321,47 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            // K-major Q/K operands: leading offset 16 B (unused under the 128-byte
+            // swizzle), 8-row groups 1024 B apart.  MN-major V: the two 64-wide
+            // halves of D are one region (RB) apart, 8-key groups 1024 B apart.
+            constexpr uint32_t kDescHiK = smem_desc_hi(1024), kDescHiV = smem_desc_hi(1024);
+            const uint32_t qdesc_lo = smem_desc_lo(sQ, 16);
+            const uint32_t kdesc_lo = smem_desc_lo(sK, 16);
+            const uint32_t vdesc_lo = smem_desc_lo(sV, RB);
             uint32_t kc = 0, vc = 0, uc = 0;
             uint32_t pc[2] = {0, 0};
             bool ok = true;
             for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++uc) {
                 const UnitPlan P = plan_unit(p, u);
                 const int n = P.n;
-                if (!mbar_wait_bounded(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
-                // S_t = Q_t K^T for key tile j, into tensor-memory columns [t*128, t*128+128)
+                if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
+                // S_t = Q_t K^T for key tile j, into tensor-memory columns [t*128, t*128+128).
+                // Descriptors step along K by adding to their low word only.
                 auto issue_s = [&](int t, uint32_t kslot) {
-                    const uint32_t qa = sQ + t * TB, kb = sK + kslot * TB;
+                    const uint32_t alo = qdesc_lo + t * (TB >> 4), blo = kdesc_lo + kslot * (TB >> 4);
+                    const uint32_t d = tmem + t * 128;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * RB + (kk & 3) * 32;
-                        mma_ss(tmem + t * 128, make_smem_desc(qa + off, 16, 1024),
-                               make_smem_desc(kb + off, 16, 1024), Cfg::IDESC_QK, kk > 0);
+                        const uint32_t off = ((kk >> 2) * RB + (kk & 3) * 32) >> 4;
+                        mma_ss(d, smem_desc64(alo + off, kDescHiK), smem_desc64(blo + off, kDescHiK),
+                               Cfg::IDESC_QK, kk > 0);
                     }
                 };
-                // O_t (+)= P_t V, P_t read from tensor memory over S_t's columns
-                auto issue_pv = [&](int t, uint32_t vslot, bool acc) {
-                    const uint32_t vb = sV + vslot * TB;
+                // O_t (+)= P_t V for keys [64*half, 64*half+64), P_t read from tensor
+                // memory over S_t's columns
+                auto issue_pv = [&](int t, uint32_t vslot, bool acc, int half) {
+                    const uint32_t blo = vdesc_lo + vslot * (TB >> 4);
+                    const uint32_t d = tmem + 256 + t * 128, a = tmem + t * 128;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                               make_smem_desc(vb + kk * 16 * 128, RB, 1024), Cfg::IDESC_PV,
-                               (acc || kk > 0) ? 1u : 0u);
+                    for (int k4 = 0; k4 < BN / 32; ++k4) {
+                        const int kk = half * (BN / 32) + k4;
+                        mma_ts(d, a + kk * 8, smem_desc64(blo + ((kk * 16 * 128) >> 4), kDescHiV),
+                               Cfg::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
                     }
                 };
                 {   // prologue: S for tile 0
                     const uint32_t ks = kc % KST, kph = (kc / KST) & 1;
-                    if (!mbar_wait_bounded(bar_k_full + 8 * ks, kph, abort_flag, limit)) { ok = false; break; }
+                    if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_k_full + 8 * ks, kph, abort_flag, limit)) { ok = false; break; }
                     tc_fence_after();
                     issue_s(0, ks);
                     mma_commit(bar_s_full);
@@ -354,27 +375,39 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 for (int j = 0; j < n && ok; ++j) {
                     const uint32_t vs = vc % VST, vph = (vc / VST) & 1;
-                    if (!mbar_wait_bounded(bar_v_full + 8 * vs, vph, abort_flag, limit)) { ok = false; break; }
-                    if (!mbar_wait_bounded(bar_p_full, pc[0] & 1, abort_flag, limit)) { ok = false; break; }
+                    if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_v_full + 8 * vs, vph, abort_flag, limit)) { ok = false; break; }
+                    if (Cfg::kSplitPV) {
+                        if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_p_half, pc[0] & 1, abort_flag, limit)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(0, vs, j > 0, 0);
+                    }
+                    if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_p_full, pc[0] & 1, abort_flag, limit)) { ok = false; break; }
                     ++pc[0];
                     tc_fence_after();
-                    issue_pv(0, vs, j > 0);
+                    if (!Cfg::kSplitPV) issue_pv(0, vs, j > 0, 0);
+                    issue_pv(0, vs, j > 0, 1);
                     if (j == n - 1) mma_commit(bar_o_full);
                     uint32_t ks = 0;
                     const bool more = (j + 1 < n);
                     if (more) {
                         ks = kc % KST;
                         const uint32_t kph = (kc / KST) & 1;
-                        if (!mbar_wait_bounded(bar_k_full + 8 * ks, kph, abort_flag, limit)) { ok = false; break; }
+                        if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_k_full + 8 * ks, kph, abort_flag, limit)) { ok = false; break; }
                         tc_fence_after();
                         issue_s(0, ks);
                         mma_commit(bar_s_full);
                     }
                     if (P.act1) {
-                        if (!mbar_wait_bounded(bar_p_full + 8, pc[1] & 1, abort_flag, limit)) { ok = false; break; }
+                        if (Cfg::kSplitPV) {
+                            if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_p_half + 8, pc[1] & 1, abort_flag, limit)) { ok = false; break; }
+                            tc_fence_after();
+                            issue_pv(1, vs, j > 0, 0);
+                        }
+                        if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_p_full + 8, pc[1] & 1, abort_flag, limit)) { ok = false; break; }
                         ++pc[1];
                         tc_fence_after();
-                        issue_pv(1, vs, j > 0);
+                        if (!Cfg::kSplitPV) issue_pv(1, vs, j > 0, 0);
+                        issue_pv(1, vs, j > 0, 1);
                         if (j == n - 1) mma_commit(bar_o_full + 8);
                     }
                     mma_commit(bar_v_empty + 8 * vs);
@@ -453,12 +486,21 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 float mx[8];
+                if constexpr (Cfg::kMax3) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mx[e] = s[e];
+                    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(s[e], s[8 + e]);
 #pragma unroll
-                for (int c = 8; c < BN; c += 8)
+                    for (int c = 16; c < BN; c += 16)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
+                        for (int e = 0; e < 8; ++e) mx[e] = fmax3f(mx[e], s[c + e], s[c + 8 + e]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+                    for (int c = 8; c < BN; c += 8)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
+                }
                 const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                 const float m_tile = mt * sl2;
@@ -503,6 +545,13 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         pk[e] = pack_bf16x2(pe.x, pe.y);
                     }
                     tmem_st16(tS + c * 16, pk);
+                    if (Cfg::kSplitPV && c == BN / 64 - 1) {
+                        // first half of P (keys 0..63) is in place: let its PV start
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_p_half + 8 * t);
+                    }
                 }
                 const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
                 const float2 asum = fadd2(a01, a23);
