@@ -262,17 +262,27 @@ def run_native(args):
     kv_bytes = int(L.sum().item()) * dw.Hkv * dw.D * 2 * 2     # K and V rows read, all steps
     other_bytes = dw.steps * dw.B * (2 * dw.Hq * dw.D * 2 + 2 * 2 * dw.Hkv * dw.D * 2)  # q, out, append r+w
 
-    def decode_all():
+    # events around every swa_decode call (split-KV kernel + split merge) are
+    # captured into the graph, so each replay re-records them on the launch stream
+    dec_ev = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True))
+              for _ in range(dw.steps)]
+
+    def decode_all(with_events=False):
         for s in range(dw.steps):
             swa.swa_cache_append(d_kn[s], d_vn[s], d_kc, d_vc, d_pos[s])
+            if with_events:
+                dec_ev[s][0].record()
             swa.swa_decode(d_q[s], d_kc, d_vc, d_pos[s], dw.scale, out=d_out[s], workspace=d_ws)
+            if with_events:
+                dec_ev[s][1].record()
 
     # ---- capture the 128 decode steps in one graph
     decode_all()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        decode_all()
+        decode_all(with_events=True)
     torch.cuda.synchronize()
 
     def step(ev=None):
@@ -307,6 +317,8 @@ def run_native(args):
         torch.cuda.synchronize()
     barrier(world)
     status = swa.swa_get_device_status()
+    # decode launches of the last timed replay (128 calls)
+    dec_call_ms = sum(a.elapsed_time(b) for a, b in dec_ev)
     pf_ms = [e[0].elapsed_time(e[1]) for e in evs]
     ch_ms = [e[1].elapsed_time(e[2]) for e in evs]
     de_ms = [e[2].elapsed_time(e[3]) for e in evs]
@@ -324,6 +336,12 @@ def run_native(args):
     dec_tok_s = weak_scaling_rate(dw.B * dw.steps * args.steps, world, de_total * 1e-3)
     dec_gbs = (kv_bytes + other_bytes) / ((de_total / args.steps) * 1e-3) / 1e9
     dec_kv_gbs = kv_bytes / ((de_total / args.steps) * 1e-3) / 1e9
+    # roofline of the dominant launch (decode: split-KV kernel + merge), bytes
+    # it must move per call (K/V rows in the window, q in, out back) over the
+    # event-timed duration of the calls
+    dec_call_ms = max_over_ranks(dec_call_ms, world)
+    dec_call_bytes = kv_bytes + dw.steps * dw.B * 2 * dw.Hq * dw.D * 2
+    dec_call_gbs = dec_call_bytes / (dec_call_ms * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers
     hq, hk, hv = q_cpu.pin_memory(), k_cpu.pin_memory(), v_cpu.pin_memory()
@@ -384,6 +402,19 @@ def run_native(args):
                 "step": "one-shot prefill + 4-chunk prefill (N=16384) + 128 decode steps (B=64, graph)",
             },
             "roofline": {
+                "bound": "hbm",
+                "kernel": "swa_decode (swa_decode_kernel<128,4> + swa_decode_combine_kernel<128,4>)",
+                "why_this_kernel": "largest share of the step's GPU time (ncu launch list and events)",
+                "achieved": dec_call_gbs,
+                "peak": peaks["hbm_gbs"],
+                "unit": "GB/s",
+                "frac": dec_call_gbs / peaks["hbm_gbs"],
+                "peak_kind": f"HBM copy ({peaks['source']})",
+                "traffic": ncu_traffic("swa_decode_kernel<128,4>"),
+                "algorithmic_bytes_per_launch": dec_call_bytes / dw.steps,
+                "avg_launch_us": dec_call_ms * 1e3 / dw.steps,
+            },
+            "roofline_prefill": {
                 "bound": "tensor",
                 "kernel": "swa_prefill_kernel<128>",
                 "achieved": achieved,

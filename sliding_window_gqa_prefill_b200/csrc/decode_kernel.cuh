@@ -375,7 +375,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 
 // Log-sum-exp merge of the splits of each (sequence, kv head) into bf16 out.
 template <int D, int G>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(1024)
 swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restrict__ ws_ml,
                           const float *__restrict__ ws_o, __nv_bfloat16 *__restrict__ out,
                           int Hkv, int W, int nsplit_max) {

@@ -166,7 +166,7 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
         Hkv, W, nsm, scale * kLog2e);
     SWA_CUDA_TRY(cudaGetLastError());
     if (nsm > 1) {
-        swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), 128, 0, s>>>(
+        swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), G * D, 0, s>>>(
             pos, ws_ml, ws_o, static_cast<__nv_bfloat16 *>(out), Hkv, W, nsm);
         SWA_CUDA_TRY(cudaGetLastError());
     }

@@ -38,7 +38,9 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     assert torch.cuda.is_available()
     swa.build()
     L = swa.lib()
-    B, Hq, Hkv, D, W = 16, 32, 8, 128, 4096
+    # W = 8192: 16 splits of 512 keys per sequence, merged through the scratch
+    B, Hq, Hkv, D, W = 16, 32, 8, 128, 8192
+    assert swa.swa_decode_workspace_size(B, Hq, Hkv, D, W) > 0
     scale = 1.0 / math.sqrt(D)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call, seed in enumerate((101, 202)):
@@ -64,7 +66,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     swa.build()
     L = swa.lib()
-    B, Hq, Hkv, D, W = 512, 32, 8, 128, 4096          # needs ~68 MB of partials
+    B, Hq, Hkv, D, W = 256, 32, 8, 128, 8192          # needs ~68 MB of partials
     assert swa.swa_decode_workspace_size(B, Hq, Hkv, D, W) > (16 << 20)
     st = L.swa_decode_noalloc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, B, Hq, Hkv, D, W, 0.1, None)
     assert st == swa.SWA_ERR_UNSUPPORTED
