@@ -54,6 +54,8 @@ def _load():
             lib.oracle_slot_positions.argtypes = [ip, i, i, ip]
             lib.oracle_swa_chunk.argtypes = [dp, dp, dp, dp, dp, ip, ip, dp, i, i, i, i, i, i, d, i]
             lib.oracle_swa_decode.argtypes = [dp, dp, dp, ip, ip, dp, i, i, i, i, i, d, i]
+            lib.oracle_rope.argtypes = [dp, ip, i, i, i, i, d]
+            lib.oracle_rope.restype = ctypes.c_int
             for f in (lib.oracle_swa_prefill, lib.oracle_cache_append, lib.oracle_slot_positions,
                       lib.oracle_swa_chunk, lib.oracle_swa_decode):
                 f.restype = ctypes.c_int
@@ -182,3 +184,15 @@ def swa_decode(q, k_cache, v_cache, slot_pos, pos, W: int, scale: float,
     if rc != 0:
         raise ValueError("oracle_swa_decode: bad arguments")
     return out
+
+
+def rope(x, pos, theta: float = 10000.0) -> np.ndarray:
+    """Rotary embedding of x [B, T, H, D] at positions pos[b] + t (adjacent
+    pairs, angle p * theta^(-2i/D)); returns a new float64 array."""
+    y = _f64(x).copy()
+    p = _i32(pos)
+    B, T, H, D = y.shape
+    rc = _load().oracle_rope(_dp(y), _ip(p), B, T, H, D, float(theta))
+    if rc != 0:
+        raise ValueError("oracle_rope: bad arguments")
+    return y

@@ -130,6 +130,32 @@ int oracle_swa_prefill(const double *q, const double *k, const double *v,
     return bad ? -1 : 0;
 }
 
+/* Rotary position embedding, in place (the pages give only its base:
+ * "RoPE theta=10000" in Table 1 of [P1] "Methods").  Adopted reading: the
+ * rotary embedding of Su et al. (RoFormer) in its original pairing, adjacent
+ * elements (2i, 2i+1) form a pair rotated by the angle p * theta^(-2i/D):
+ *   (x0, x1) -> (x0 cos a - x1 sin a, x0 sin a + x1 cos a).
+ * x : [B, T, H, D] doubles, position of row (b, t) = pos[b] + t. */
+int oracle_rope(double *x, const int32_t *pos, int B, int T, int H, int D, double theta)
+{
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D & 1) || !(theta > 1.0)) return -1;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            const double p = (double)pos[b] + t;
+            for (int h = 0; h < H; ++h) {
+                double *row = x + (((size_t)b * T + t) * H + h) * D;
+                for (int i = 0; i < D / 2; ++i) {
+                    const double a = p * pow(theta, -2.0 * i / D);
+                    const double c = cos(a), s = sin(a);
+                    const double x0 = row[2 * i], x1 = row[2 * i + 1];
+                    row[2 * i] = x0 * c - x1 * s;
+                    row[2 * i + 1] = x0 * s + x1 * c;
+                }
+            }
+        }
+    return 0;
+}
+
 /* Rolling-buffer write ([P1] "Rolling Buffer KV Cache 동작 설명", write step;
  * [P2] section 3.3; [P4] section 3): for every sequence b and every new token
  * t, position p = pos[b] + t goes to slot p mod W.  The bytes are copied

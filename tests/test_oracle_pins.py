@@ -297,3 +297,55 @@ def test_useful_pair_counts():
     assert workloads.useful_pairs(16384, 16384) == 134_225_920
     assert abs(134_225_920 / 58_722_304 - 2.286) < 1e-3
     assert workloads.useful_flops(2, 16384, 4096, 32, 128) == 1_924_212_457_472
+
+
+# ---------------------------------------------------------------- rotary position embedding
+
+def test_rope_position_zero_is_identity(oracle_mod):
+    x = _rand((2, 1, 3, 16), 40)
+    np.testing.assert_array_equal(oracle_mod.rope(x, [0, 0]), x)
+
+
+def test_rope_closed_form_two_dims(oracle_mod):
+    """D = 2: the single pair turns by p radians (theta^0 = 1)."""
+    x = np.zeros((1, 5, 1, 2))
+    x[..., 0] = 1.0
+    y = oracle_mod.rope(x, [3])
+    for t in range(5):
+        np.testing.assert_allclose(y[0, t, 0], [np.cos(3 + t), np.sin(3 + t)], rtol=0, atol=1e-15)
+
+
+def test_rope_matches_complex_multiplication(oracle_mod):
+    """Brute force with numpy complex numbers: pair i is the complex number
+    x[2i] + 1j*x[2i+1], multiplied by exp(1j * p * theta**(-2i/D))."""
+    B, T, H, D = 2, 7, 3, 64
+    x = _rand((B, T, H, D), 41)
+    pos = [5, 31000]
+    y = oracle_mod.rope(x, pos)
+    c = x[..., 0::2] + 1j * x[..., 1::2]
+    p = (np.asarray(pos)[:, None] + np.arange(T)[None, :]).astype(np.float64)
+    ang = p[:, :, None, None] * (10000.0 ** (-np.arange(D // 2) * 2.0 / D))[None, None, None, :]
+    z = c * np.exp(1j * ang)
+    np.testing.assert_allclose(y[..., 0::2], z.real, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(y[..., 1::2], z.imag, rtol=0, atol=1e-9)
+
+
+def test_rope_preserves_pair_norms_and_composes(oracle_mod):
+    x = _rand((1, 4, 2, 32), 42)
+    y = oracle_mod.rope(x, [100])
+    n0 = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    n1 = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    np.testing.assert_allclose(n1, n0, rtol=1e-12)
+    # rotating by a then by b equals rotating by a + b (one row: row t adds t twice)
+    x1 = x[:, :1]
+    z = oracle_mod.rope(oracle_mod.rope(x1, [100]), [250])
+    np.testing.assert_allclose(z, oracle_mod.rope(x1, [350]), rtol=0, atol=1e-9)
+
+
+def test_rope_scores_depend_on_relative_position_only(oracle_mod):
+    """<R(p) q, R(p') k> is unchanged when both positions shift by the same c."""
+    q = _rand((1, 1, 1, 128), 43)
+    k = _rand((1, 1, 1, 128), 44)
+    s1 = float(np.sum(oracle_mod.rope(q, [1000]) * oracle_mod.rope(k, [900])))
+    s2 = float(np.sum(oracle_mod.rope(q, [1100 + 4096]) * oracle_mod.rope(k, [1000 + 4096])))
+    assert abs(s1 - s2) < 1e-8

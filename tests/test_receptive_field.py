@@ -1,0 +1,66 @@
+"""Receptive field of stacked sliding-window layers.
+
+The pages: a token at layer k reaches k*W positions back through the stack
+("Mistral 7B -- Sliding Window Attention" summary, section "Methods"; the
+receptive-field simulator of "Mistral 7B: Engineering Extreme Efficiency in
+LLMs", section 2, prints a span of 9 tokens for W = 3 and 3 layers, formula
+Span = L x W).  With identity projections (q = k = v = the layer input) a
+stack of L SWA layers is run on a sequence; one input position j is perturbed;
+exactly the outputs at positions j .. j + L*lookback change, where lookback is
+W under the i-W <= j <= i reading (the simulator's) and W-1 under the adopted
+i-W < j <= i reading.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sliding_window_gqa_prefill_b200 import workloads as wl
+
+
+def _stack_oracle(oracle_mod, x, W, L, mode):
+    for _ in range(L):
+        x = oracle_mod.swa_prefill(x, x, x, W, 1.0 / np.sqrt(x.shape[-1]), mode=mode)
+    return x
+
+
+def _changed_positions(a, b):
+    return sorted(set(np.nonzero(np.abs(a - b).reshape(a.shape[0], a.shape[1], -1).max(axis=(0, 2)) > 0)[0].tolist()))
+
+
+@pytest.mark.parametrize("W,L,mode,span", [(3, 3, 1, 9), (3, 3, 0, 6), (5, 2, 0, 8), (4, 1, 1, 4)])
+def test_oracle_stack_reach(oracle_mod, W, L, mode, span):
+    """W=3, L=3 under the simulator's reading reaches exactly 9 positions back."""
+    rng = np.random.default_rng(W * 10 + L)
+    N, D, j = 40, 8, 11
+    x = rng.standard_normal((1, N, 1, D))
+    y = x.copy()
+    y[0, j] += 5.0 * rng.standard_normal(D)
+    a = _stack_oracle(oracle_mod, x, W, L, mode)
+    b = _stack_oracle(oracle_mod, y, W, L, mode)
+    assert _changed_positions(a, b) == list(range(j, j + span + 1))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("W,L,mode,span", [(3, 3, 1, 9), (3, 3, 0, 6), (130, 2, 0, 258)])
+def test_gpu_stack_reach(W, L, mode, span):
+    """The same on the CUDA prefill (bf16 between layers): outputs beyond the
+    reach are bit-identical, the ones inside it move."""
+    import sliding_window_gqa_prefill_b200 as swa
+    assert torch.cuda.is_available()
+    swa.build()
+    N, H, D, j = 600, 2, 64, 37
+    x = wl.random_bf16((1, N, H, D), 77).cuda()
+    y = x.clone()
+    y[0, j] = (wl.random_bf16((H, D), 78) * 20).cuda()
+
+    def stack(t):
+        for _ in range(L):
+            t = swa.swa_prefill(t, t, t, W, 1.0 / np.sqrt(D), window_mode=mode)
+        return t
+
+    a, b = stack(x), stack(y)
+    torch.cuda.synchronize()
+    diff = (a.float() - b.float()).abs().amax(dim=(0, 2, 3)).cpu().numpy()
+    changed = np.nonzero(diff > 0)[0].tolist()
+    assert changed and changed[0] == j and changed[-1] == j + span, (changed[:3], changed[-3:])
+    assert all(diff[i] == 0 for i in range(N) if i < j or i > j + span)
