@@ -170,6 +170,51 @@ swa_status_t swa_decode_noalloc(const void *q, const void *k_cache, const void *
                                 int W, float scale, swa_stream_t stream);
 
 /*
+ * Rotary position embedding (RoPE).  The pages give only its base, theta =
+ * 10000, in the Table 1 line of "Methods" of the "Mistral 7B -- Sliding
+ * Window Attention" summary.  Adopted convention (the original RoFormer
+ * pairing): adjacent elements (2i, 2i+1) of a head vector at position p turn
+ * by the angle p * theta^(-2i/D):
+ *   (x0, x1) -> (x0 cos a - x1 sin a, x0 sin a + x1 cos a).
+ * Angles are formed and reduced in double precision; the rotation runs in
+ * fp32 and rotated tensors are stored in bf16.  theta must be finite and > 1.
+ */
+
+/* swa_rope -- rotate x [B, T, H, D] (bf16, device) in place, row (b, t) at
+ * position pos[b] + t (pos: int32 [B], device). */
+swa_status_t swa_rope(void *x, const int32_t *pos, int B, int T, int H, int D, float theta,
+                      swa_stream_t stream);
+
+/* swa_cache_append_rope -- swa_cache_append that rotates the keys on their
+ * way into the cache (the cache holds rotated keys; values are copied). */
+swa_status_t swa_cache_append_rope(const void *k_new, const void *v_new, void *k_cache,
+                                   void *v_cache, const int32_t *pos, int B, int T, int Hkv,
+                                   int D, int W, float theta, swa_stream_t stream);
+
+/* swa_prefill_rope -- swa_prefill with q given unrotated: each Q tile is
+ * rotated (positions 0..N-1) in shared memory right after its TMA load.  k
+ * must already be rotated (swa_rope).  Same arguments as swa_prefill plus
+ * theta. */
+swa_status_t swa_prefill_rope(const void *q, const void *k, const void *v, void *out, int B, int N,
+                              int Hq, int Hkv, int D, int W, int window_mode, float scale,
+                              float theta, swa_stream_t stream);
+
+/* swa_prefill_chunk_rope -- swa_prefill_chunk with q given unrotated (rotated
+ * at load, positions start_pos[b] + t); the chunk's k must already be rotated
+ * and the cache holds rotated keys (swa_cache_append_rope or this call). */
+swa_status_t swa_prefill_chunk_rope(const void *q, const void *k, const void *v, void *k_cache,
+                                    void *v_cache, const int32_t *start_pos, void *out, int B,
+                                    int C, int Hq, int Hkv, int D, int W, float scale, float theta,
+                                    swa_stream_t stream);
+
+/* swa_decode_rope -- swa_decode with q given unrotated (rotated in fp32 at
+ * position pos[b] while loaded); the cache holds rotated keys. */
+swa_status_t swa_decode_rope(const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
+                             float scale, float theta, void *workspace, size_t workspace_bytes,
+                             swa_stream_t stream);
+
+/*
  * swa_get_device_status -- synchronise `stream`, then return (and reset to
  * SWA_OK) the device status word that kernels of this library set when a
  * bounded wait runs out.  Returns SWA_ERR_CUDA if synchronisation fails.

@@ -18,7 +18,7 @@ import threading
 __all__ = [
     "SwaError", "build", "lib", "swa_prefill", "swa_prefill_chunk", "swa_cache_append",
     "swa_decode", "swa_decode_workspace_size", "swa_get_device_status", "swa_set_wait_limit_ns",
-    "swa_selftest_wait_timeout", "SWA_OK", "SWA_ERR_INVALID_ARG", "SWA_ERR_UNSUPPORTED",
+    "swa_selftest_wait_timeout", "swa_rope", "SWA_OK", "SWA_ERR_INVALID_ARG", "SWA_ERR_UNSUPPORTED",
     "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_WINDOW_EXCL_LEFT", "SWA_WINDOW_INCL_LEFT",
 ]
 
@@ -80,6 +80,14 @@ def lib() -> ctypes.CDLL:
             L.swa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, ctypes.c_size_t, st]
             L.swa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, st]
             L.swa_decode_noalloc.restype = ctypes.c_int
+            L.swa_rope.argtypes = [vp, vp, i, i, i, i, f, st]
+            L.swa_cache_append_rope.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, st]
+            L.swa_prefill_rope.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, f, st]
+            L.swa_prefill_chunk_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, st]
+            L.swa_decode_rope.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, vp, ctypes.c_size_t, st]
+            for fn in (L.swa_rope, L.swa_cache_append_rope, L.swa_prefill_rope, L.swa_prefill_chunk_rope,
+                       L.swa_decode_rope):
+                fn.restype = ctypes.c_int
             L.swa_decode_workspace_size.argtypes = [i, i, i, i, i]
             L.swa_decode_workspace_size.restype = ctypes.c_size_t
             L.swa_get_device_status.argtypes = [st]
@@ -132,51 +140,83 @@ def _i32(t, name: str, n: int):
 
 
 def swa_prefill(q, k, v, W: int, scale: float, out=None, window_mode: int = SWA_WINDOW_EXCL_LEFT,
-                stream=None):
-    """One-shot SWA prefill.  q [B,N,Hq,D], k/v [B,N,Hkv,D] bf16 -> out [B,N,Hq,D]."""
+                stream=None, rope_theta: float | None = None):
+    """One-shot SWA prefill.  q [B,N,Hq,D], k/v [B,N,Hkv,D] bf16 -> out [B,N,Hq,D].
+
+    rope_theta: if given, q is unrotated and gets the rotary embedding inside
+    the kernel (swa_prefill_rope); k must already be rotated."""
     import torch
     B, N, Hq, D = q.shape
     Hkv = k.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    _check(lib().swa_prefill(_bf16(q, "q"), _bf16(k, "k", (B, N, Hkv, D)), _bf16(v, "v", (B, N, Hkv, D)),
-                             _bf16(out, "out", (B, N, Hq, D)), B, N, Hq, Hkv, D, int(W),
-                             int(window_mode), float(scale), _stream_handle(stream)), "swa_prefill")
+    args = (_bf16(q, "q"), _bf16(k, "k", (B, N, Hkv, D)), _bf16(v, "v", (B, N, Hkv, D)),
+            _bf16(out, "out", (B, N, Hq, D)), B, N, Hq, Hkv, D, int(W), int(window_mode), float(scale))
+    if rope_theta is None:
+        _check(lib().swa_prefill(*args, _stream_handle(stream)), "swa_prefill")
+    else:
+        _check(lib().swa_prefill_rope(*args, float(rope_theta), _stream_handle(stream)), "swa_prefill_rope")
     return out
 
 
 def swa_prefill_chunk(q, k, v, k_cache, v_cache, start_pos, W: int, scale: float, out=None,
-                      stream=None):
-    """Chunked prefill of one chunk through the rolling buffer (updates the cache)."""
+                      stream=None, rope_theta: float | None = None):
+    """Chunked prefill of one chunk through the rolling buffer (updates the cache).
+
+    rope_theta: if given, q is unrotated (rotated in the kernel); k must already
+    be rotated and the cache holds rotated keys (swa_prefill_chunk_rope)."""
     import torch
     B, C, Hq, D = q.shape
     Hkv = k.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    _check(lib().swa_prefill_chunk(
-        _bf16(q, "q"), _bf16(k, "k", (B, C, Hkv, D)), _bf16(v, "v", (B, C, Hkv, D)),
-        _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
-        _i32(start_pos, "start_pos", B), _bf16(out, "out", (B, C, Hq, D)), B, C, Hq, Hkv, D, int(W),
-        float(scale), _stream_handle(stream)), "swa_prefill_chunk")
+    args = (_bf16(q, "q"), _bf16(k, "k", (B, C, Hkv, D)), _bf16(v, "v", (B, C, Hkv, D)),
+            _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+            _i32(start_pos, "start_pos", B), _bf16(out, "out", (B, C, Hq, D)), B, C, Hq, Hkv, D, int(W),
+            float(scale))
+    if rope_theta is None:
+        _check(lib().swa_prefill_chunk(*args, _stream_handle(stream)), "swa_prefill_chunk")
+    else:
+        _check(lib().swa_prefill_chunk_rope(*args, float(rope_theta), _stream_handle(stream)),
+               "swa_prefill_chunk_rope")
     return out
 
 
-def swa_cache_append(k_new, v_new, k_cache, v_cache, pos, stream=None) -> None:
-    """Write k_new/v_new [B,T,Hkv,D] at slots (pos[b]+t) mod W of the caches [B,W,Hkv,D]."""
+def swa_cache_append(k_new, v_new, k_cache, v_cache, pos, stream=None,
+                     rope_theta: float | None = None) -> None:
+    """Write k_new/v_new [B,T,Hkv,D] at slots (pos[b]+t) mod W of the caches [B,W,Hkv,D].
+
+    rope_theta: if given, the keys are rotated on the way in (swa_cache_append_rope)."""
     B, T, Hkv, D = k_new.shape
     W = k_cache.shape[1]
-    _check(lib().swa_cache_append(
-        _bf16(k_new, "k_new"), _bf16(v_new, "v_new", (B, T, Hkv, D)),
-        _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
-        _i32(pos, "pos", B), B, T, Hkv, D, W, _stream_handle(stream)), "swa_cache_append")
+    args = (_bf16(k_new, "k_new"), _bf16(v_new, "v_new", (B, T, Hkv, D)),
+            _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+            _i32(pos, "pos", B), B, T, Hkv, D, W)
+    if rope_theta is None:
+        _check(lib().swa_cache_append(*args, _stream_handle(stream)), "swa_cache_append")
+    else:
+        _check(lib().swa_cache_append_rope(*args, float(rope_theta), _stream_handle(stream)),
+               "swa_cache_append_rope")
+
+
+def swa_rope(x, pos, theta: float = 10000.0, stream=None):
+    """Rotate x [B,T,H,D] (bf16, CUDA) in place at positions pos[b]+t; returns x."""
+    B, T, H, D = x.shape
+    _check(lib().swa_rope(_bf16(x, "x"), _i32(pos, "pos", B), B, T, H, D, float(theta),
+                          _stream_handle(stream)), "swa_rope")
+    return x
 
 
 def swa_decode_workspace_size(B: int, Hq: int, Hkv: int, D: int, W: int) -> int:
     return int(lib().swa_decode_workspace_size(B, Hq, Hkv, D, W))
 
 
-def swa_decode(q, k_cache, v_cache, pos, scale: float, out=None, workspace=None, stream=None):
-    """Decode one token per sequence.  q [B,Hq,D]; caches [B,W,Hkv,D]; pos int32 [B]."""
+def swa_decode(q, k_cache, v_cache, pos, scale: float, out=None, workspace=None, stream=None,
+               rope_theta: float | None = None):
+    """Decode one token per sequence.  q [B,Hq,D]; caches [B,W,Hkv,D]; pos int32 [B].
+
+    rope_theta: if given, q is unrotated and rotated at pos[b] in the kernel
+    (swa_decode_rope); the cache must hold rotated keys."""
     import torch
     B, Hq, D = q.shape
     W, Hkv = k_cache.shape[1], k_cache.shape[2]
@@ -185,11 +225,13 @@ def swa_decode(q, k_cache, v_cache, pos, scale: float, out=None, workspace=None,
     need = swa_decode_workspace_size(B, Hq, Hkv, D, W)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    _check(lib().swa_decode(
-        _bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
-        _i32(pos, "pos", B), _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale),
-        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-        _stream_handle(stream)), "swa_decode")
+    head = (_bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+            _i32(pos, "pos", B), _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale))
+    tail = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if rope_theta is None:
+        _check(lib().swa_decode(*head, *tail), "swa_decode")
+    else:
+        _check(lib().swa_decode_rope(*head, float(rope_theta), *tail), "swa_decode_rope")
     return out
 
 

@@ -101,7 +101,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kc,
                   const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ pos,
                   __nv_bfloat16 *__restrict__ out, float2 *__restrict__ ws_ml,
-                  float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2) {
+                  float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2,
+                  int rope, const RopeTable rope_freq) {
     using Cfg = DecodeCfg<D, G>;
     constexpr int LPR = Cfg::LPR, KPR = Cfg::KPR, KI = Cfg::KI, NV = Cfg::NV;
     constexpr int TLEV = Cfg::TLEV, VPL = Cfg::VPL;
@@ -134,6 +135,16 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)b * Hq + g * G + h) * D) + sub);
         float qf[8];
         bf16x8_to_f32(raw, qf);
+        if (rope) {            // rotary embedding of the query at its position, in fp32
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float c, sn;
+                rope_cos_sin((double)p, rope_freq.f[sub * 4 + e], c, sn);
+                const float x0 = qf[2 * e], x1 = qf[2 * e + 1];
+                qf[2 * e] = x0 * c - x1 * sn;
+                qf[2 * e + 1] = x0 * sn + x1 * c;
+            }
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) q2[h][e] = make_float2(qf[2 * e] * scale_log2, qf[2 * e + 1] * scale_log2);
     }
@@ -430,10 +441,12 @@ swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restr
 // Rolling-buffer write: cache[b, (pos[b]+t) mod W, h, :] = new[b, t, h, :],
 // 16-byte copies, grid-stride over every (b, t, h, 16-byte chunk) of K and V.
 // Write step of "Rolling Buffer KV Cache 동작 설명" (slot = p % W).
+// With rope != 0 the keys are rotated (rotary embedding at their position)
+// on the way into the cache; values are copied unchanged.
 __global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                                   uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                                   const int32_t *__restrict__ pos, int B, int T, int W,
-                                  int row_vec) {
+                                  int row_vec, int head_vec, int rope, const RopeTable rope_freq) {
     // row_vec = Hkv*D*2/16 sixteen-byte vectors per (b, t) row
     const long long total = (long long)B * T * row_vec;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -450,8 +463,34 @@ __global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *
         const long long p = (long long)p0 + t;
         const int slot = (int)(p % W);
         const size_t dst = ((size_t)b * W + slot) * row_vec + c;
-        k_cache[dst] = __ldg(k_new + i);
+        uint4 kv = __ldg(k_new + i);
+        if (rope) kv = rope_rotate8(kv, (c % head_vec) * 4, (double)p, rope_freq);
+        k_cache[dst] = kv;
         v_cache[dst] = __ldg(v_new + i);
+    }
+}
+
+}  // namespace swa
+
+namespace swa {
+
+// In-place rotary embedding of x [B, T, H, D] (bf16), row (b, t) at position
+// pos[b] + t; 16-byte words of four adjacent pairs, grid-stride.
+__global__ void swa_rope_kernel(uint4 *__restrict__ x, const int32_t *__restrict__ pos, int B, int T,
+                                int row_vec, int head_vec, const RopeTable rope_freq) {
+    const long long total = (long long)B * T * row_vec;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int c = (int)(i % row_vec);
+        const long long bt = i / row_vec;
+        const int t = (int)(bt % T);
+        const int b = (int)(bt / T);
+        const int p0 = __ldg(pos + b);
+        if (p0 < 0) {
+            record_status(kStatusInvalid);
+            continue;
+        }
+        x[i] = rope_rotate8(x[i], (c % head_vec) * 4, (double)p0 + t, rope_freq);
     }
 }
 

@@ -53,6 +53,8 @@ struct PrefillParams {
     int chunk_mode;   // 1: keys also come from the rolling-buffer cache
     const int32_t *start_pos;  // chunk mode: [B] first position of the chunk
     __nv_bfloat16 *out;        // [B, Nq, Hq, D]
+    int rope;                  // 1: rotate each Q tile in shared memory after its load
+    RopeTable rope_freq;       // theta^(-2i/D), i < D/2
 };
 
 template <int D>
@@ -69,8 +71,8 @@ struct PrefillCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST],
-    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain, p_half[2]
-    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2;
+    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain, p_half[2], q_rot[2]
+    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-byte alignment
@@ -192,6 +194,21 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPl
     return t;
 }
 
+// Rotary embedding of row `row` of a K-major, 128-byte-swizzled bf16 tile in
+// shared memory (the layout TMA writes): 16-byte chunk c of the row in a
+// 64-column region sits at chunk c ^ (row mod 8).
+template <int D>
+__device__ __forceinline__ void rope_row_swizzled(uint8_t *tile, int row, double p, const RopeTable &tab) {
+#pragma unroll
+    for (int reg = 0; reg < D / 64; ++reg) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4 *ptr = reinterpret_cast<uint4 *>(tile + reg * 128 * 128 + row * 128 + ((c ^ (row & 7)) * 16));
+            *ptr = rope_rotate8(*ptr, reg * 32 + c * 4, p, tab);
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(384, 1)
 swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -223,6 +240,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t bar_o_full = bar_p_full + 16;
     const uint32_t bar_drain = bar_o_full + 16;
     const uint32_t bar_p_half = bar_drain + 8;                // + 8*t
+    const uint32_t bar_q_rot = bar_p_half + 16;               // + 8*t (RoPE on Q done)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::OFF_MISC + 4);
 
@@ -249,6 +267,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(bar_drain, 1);
         mbar_init(bar_p_half, 4);
         mbar_init(bar_p_half + 8, 4);
+        mbar_init(bar_q_rot, 4);
+        mbar_init(bar_q_rot + 8, 4);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -330,11 +350,24 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t vdesc_lo = smem_desc_lo(sV, RB);
             uint32_t kc = 0, vc = 0, uc = 0;
             uint32_t pc[2] = {0, 0};
+            uint32_t qr1 = 0;                      // units with a second query head
             bool ok = true;
             for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++uc) {
                 const UnitPlan P = plan_unit(p, u);
                 const int n = P.n;
                 if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
+                if (p.rope) {       // the softmax warpgroups rotate Q in place first
+                    if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_rot, uc & 1, abort_flag, limit)) { ok = false; break; }
+                    // head 1 of a pair is absent in some units (odd group size): its
+                    // barrier completes once per unit where it is present
+                    if (P.act1) {
+                        if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_rot + 8, qr1 & 1, abort_flag, limit)) {
+                            ok = false;
+                            break;
+                        }
+                        ++qr1;
+                    }
+                }
                 // S_t = Q_t K^T for key tile j, into tensor-memory columns [t*128, t*128+128).
                 // Descriptors step along K by adding to their low word only.
                 auto issue_s = [&](int t, uint32_t kslot) {
@@ -438,12 +471,24 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t tS = tmem + lane_off + t * 128;
         const uint32_t tO = tmem + lane_off + 256 + t * 128;
         const float sl2 = p.scale_log2;
-        uint32_t sc = 0, oc = 0;
+        uint32_t sc = 0, oc = 0, qc = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++qc) {
             const UnitPlan P = plan_unit(p, u);
             if (t == 1 && !P.act1) continue;
             const int i_rel = P.q0 + row;                  // query row in the q tensor
+            if (p.rope) {
+                // rotary embedding of this thread's Q row, in shared memory, at
+                // position s0 + i_rel; then make it visible to the tensor core
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_q_full, qc & 1, abort_flag, limit))) {
+                    ok = false;
+                    break;
+                }
+                rope_row_swizzled<D>(smem + Cfg::OFF_Q + t * TB, row, (double)(P.s0 + i_rel), p.rope_freq);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_q_rot + 8 * t);
+            }
             float m_use = -INFINITY, l = 0.f;
             for (int j = 0; j < P.n; ++j) {
                 const TileRef T = tile_ref(p, P, j);

@@ -134,7 +134,7 @@ swa_status_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const 
 
 swa_status_t launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
                            const int32_t *pos, int B, int T, int Hkv, int D, int W, int sms,
-                           cudaStream_t s) {
+                           const swa::RopeTable *rope, cudaStream_t s) {
     const int row_vec = Hkv * D * 2 / 16;
     const long long total = (long long)B * T * row_vec;
     long long blocks = (total + 255) / 256;
@@ -143,7 +143,8 @@ swa_status_t launch_append(const void *k_new, const void *v_new, void *k_cache, 
     if (blocks < 1) blocks = 1;
     swa::swa_append_kernel<<<(int)blocks, 256, 0, s>>>(
         static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
-        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), pos, B, T, W, row_vec);
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), pos, B, T, W, row_vec, D / 8,
+        rope ? 1 : 0, rope ? *rope : swa::RopeTable{});
     SWA_CUDA_TRY(cudaGetLastError());
     return SWA_OK;
 }
@@ -153,7 +154,7 @@ int decode_nsplit_max(int W) { return (W + swa::kDecodeSplit - 1) / swa::kDecode
 template <int D, int G>
 swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, const int32_t *pos,
                               void *out, int B, int Hkv, int W, float scale, void *ws,
-                              cudaStream_t s) {
+                              const swa::RopeTable *rope, cudaStream_t s) {
     const int nsm = decode_nsplit_max(W);
     const size_t o_elems = (size_t)B * Hkv * nsm * G * D;
     float *ws_o = static_cast<float *>(ws);
@@ -163,7 +164,7 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
     swa::swa_decode_kernel<D, G><<<grid, swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
         static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
-        Hkv, W, nsm, scale * kLog2e);
+        Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{});
     SWA_CUDA_TRY(cudaGetLastError());
     if (nsm > 1) {
         swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), G * D, 0, s>>>(
@@ -176,12 +177,12 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
 template <int D>
 swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *vc,
                              const int32_t *pos, void *out, int B, int Hkv, int W, float scale,
-                             void *ws, cudaStream_t s) {
+                             void *ws, const swa::RopeTable *rope, cudaStream_t s) {
     switch (G) {
-        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
-        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
-        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
-        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, s);
+        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
+        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
+        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
+        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
         default: return SWA_ERR_UNSUPPORTED;
     }
 }
@@ -234,13 +235,20 @@ __global__ void swa_selftest_exp2_kernel(const float *x, float *y, int n) {
     }
 }
 
-}  // namespace
+// ----------------------------------------------------------------- implementations
+// `rope` null: no rotary embedding; otherwise the frequency table.
 
-extern "C" {
+bool bad_theta(float theta) { return !(std::isfinite(theta) && theta > 1.f); }
 
-swa_status_t swa_prefill(const void *q, const void *k, const void *v, void *out, int B, int N,
-                         int Hq, int Hkv, int D, int W, int window_mode, float scale,
-                         swa_stream_t stream) {
+swa::RopeTable make_rope_table(float theta, int D) {
+    swa::RopeTable t{};
+    for (int i = 0; i < D / 2 && i < 64; ++i) t.f[i] = std::pow((double)theta, -2.0 * i / D);
+    return t;
+}
+
+swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out, int B, int N,
+                          int Hq, int Hkv, int D, int W, int window_mode, float scale,
+                          const swa::RopeTable *rope, cudaStream_t s) {
     if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
     if (B < 1 || N < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
@@ -276,14 +284,16 @@ swa_status_t swa_prefill(const void *q, const void *k, const void *v, void *out,
     p.chunk_mode = 0;
     p.start_pos = nullptr;
     p.out = static_cast<__nv_bfloat16 *>(out);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    p.rope = rope ? 1 : 0;
+    if (rope) p.rope_freq = *rope;
     return D == 128 ? launch_prefill<128>(mq, mk, mv, mk, mv, p, dev->sms, s)
                     : launch_prefill<64>(mq, mk, mv, mk, mv, p, dev->sms, s);
 }
 
-swa_status_t swa_prefill_chunk(const void *q, const void *k, const void *v, void *k_cache,
-                               void *v_cache, const int32_t *start_pos, void *out, int B, int C,
-                               int Hq, int Hkv, int D, int W, float scale, swa_stream_t stream) {
+swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, void *k_cache,
+                                void *v_cache, const int32_t *start_pos, void *out, int B, int C,
+                                int Hq, int Hkv, int D, int W, float scale,
+                                const swa::RopeTable *rope, cudaStream_t s) {
     if (!q || !k || !v || !k_cache || !v_cache || !start_pos || !out) return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
         !aligned16(v_cache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
@@ -319,17 +329,18 @@ swa_status_t swa_prefill_chunk(const void *q, const void *k, const void *v, void
     p.chunk_mode = 1;
     p.start_pos = start_pos;
     p.out = static_cast<__nv_bfloat16 *>(out);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    p.rope = rope ? 1 : 0;
+    if (rope) p.rope_freq = *rope;
     swa_status_t e = D == 128 ? launch_prefill<128>(mq, mk, mv, mkc, mvc, p, dev->sms, s)
                               : launch_prefill<64>(mq, mk, mv, mkc, mvc, p, dev->sms, s);
     if (e) return e;
-    // attend first, then write the chunk into the buffer (stream order)
-    return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, s);
+    // attend first, then write the chunk (its keys already rotated) into the buffer
+    return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, nullptr, s);
 }
 
-swa_status_t swa_cache_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                              const int32_t *pos, int B, int T, int Hkv, int D, int W,
-                              swa_stream_t stream) {
+swa_status_t append_impl(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                         const int32_t *pos, int B, int T, int Hkv, int D, int W,
+                         const swa::RopeTable *rope, cudaStream_t s) {
     if (!k_new || !v_new || !k_cache || !v_cache || !pos) return SWA_ERR_INVALID_ARG;
     if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
         (reinterpret_cast<uintptr_t>(pos) & 3u))
@@ -338,11 +349,10 @@ swa_status_t swa_cache_append(const void *k_new, const void *v_new, void *k_cach
     if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
     DeviceInfo *dev = nullptr;
     if (swa_status_t e = device_info(&dev)) return e;
-    return launch_append(k_new, v_new, k_cache, v_cache, pos, B, T, Hkv, D, W, dev->sms,
-                         reinterpret_cast<cudaStream_t>(stream));
+    return launch_append(k_new, v_new, k_cache, v_cache, pos, B, T, Hkv, D, W, dev->sms, rope, s);
 }
 
-size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W) {
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
     if (B < 1 || W < 1 || check_heads(Hq, Hkv, D) != SWA_OK) return 0;
     const size_t nsm = (size_t)decode_nsplit_max(W);
     const size_t rows = (size_t)B * Hq * nsm;        // (b, kv head, split, head in group)
@@ -350,49 +360,144 @@ size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W) {
     return o_bytes + rows * 8;
 }
 
-swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
-                        const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
-                        float scale, void *workspace, size_t workspace_bytes,
-                        swa_stream_t stream) {
+swa_status_t decode_checks(const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *pos, const void *out, int B, int Hq, int Hkv, int D,
+                           int W, float scale) {
     if (!q || !k_cache || !v_cache || !pos || !out) return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(pos) & 3u))
         return SWA_ERR_INVALID_ARG;
     if (B < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
     if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
-    const size_t need = swa_decode_workspace_size(B, Hq, Hkv, D, W);
+    if (B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+    return SWA_OK;
+}
+
+swa_status_t decode_launch(const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
+                           float scale, void *workspace, const swa::RopeTable *rope, cudaStream_t s) {
+    const int G = Hq / Hkv;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, rope, s)
+                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, rope, s);
+}
+
+swa_status_t decode_impl(const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
+                         float scale, void *workspace, size_t workspace_bytes,
+                         const swa::RopeTable *rope, cudaStream_t s) {
+    if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
+    const size_t need = decode_workspace_bytes(B, Hq, Hkv, D, W);
     if (decode_nsplit_max(W) > 1) {
         if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
     }
-    if (B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
-    const int G = Hq / Hkv;
-    DeviceInfo *dev = nullptr;
-    if (swa_status_t e = device_info(&dev)) return e;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, s)
-                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, s);
+    return decode_launch(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale, workspace, rope, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+swa_status_t swa_prefill(const void *q, const void *k, const void *v, void *out, int B, int N,
+                         int Hq, int Hkv, int D, int W, int window_mode, float scale,
+                         swa_stream_t stream) {
+    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, window_mode, scale, nullptr,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_prefill_chunk(const void *q, const void *k, const void *v, void *k_cache,
+                               void *v_cache, const int32_t *start_pos, void *out, int B, int C,
+                               int Hq, int Hkv, int D, int W, float scale, swa_stream_t stream) {
+    return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, C, Hq, Hkv, D, W, scale,
+                              nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_cache_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                              const int32_t *pos, int B, int T, int Hkv, int D, int W,
+                              swa_stream_t stream) {
+    return append_impl(k_new, v_new, k_cache, v_cache, pos, B, T, Hkv, D, W, nullptr,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W) {
+    return decode_workspace_bytes(B, Hq, Hkv, D, W);
+}
+
+swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
+                        float scale, void *workspace, size_t workspace_bytes,
+                        swa_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale, workspace,
+                       workspace_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 swa_status_t swa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
                                 const int32_t *pos, void *out, int B, int Hq, int Hkv, int D,
                                 int W, float scale, swa_stream_t stream) {
-    if (!q || !k_cache || !v_cache || !pos || !out) return SWA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(pos) & 3u))
-        return SWA_ERR_INVALID_ARG;
-    if (B < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
-    if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
-    if (swa_decode_workspace_size(B, Hq, Hkv, D, W) > kNoallocScratchBytes) return SWA_ERR_UNSUPPORTED;
-    if (B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+    if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
+    if (decode_workspace_bytes(B, Hq, Hkv, D, W) > kNoallocScratchBytes) return SWA_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     if (swa_status_t e = noalloc_scratch(&scratch)) return e;
+    return decode_launch(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale, scratch, nullptr,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_rope(void *x, const int32_t *pos, int B, int T, int H, int D, float theta,
+                      swa_stream_t stream) {
+    if (!x || !pos || !aligned16(x) || (reinterpret_cast<uintptr_t>(pos) & 3u)) return SWA_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || bad_theta(theta)) return SWA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
     DeviceInfo *dev = nullptr;
     if (swa_status_t e = device_info(&dev)) return e;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int G = Hq / Hkv;
-    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, scratch, s)
-                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, scratch, s);
+    const swa::RopeTable tab = make_rope_table(theta, D);
+    const int row_vec = H * D / 8, head_vec = D / 8;
+    const long long total = (long long)B * T * row_vec;
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)dev->sms * 16) blocks = (long long)dev->sms * 16;
+    swa::swa_rope_kernel<<<(int)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4 *>(x), pos, B, T, row_vec, head_vec, tab);
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
+}
+
+swa_status_t swa_cache_append_rope(const void *k_new, const void *v_new, void *k_cache,
+                                   void *v_cache, const int32_t *pos, int B, int T, int Hkv,
+                                   int D, int W, float theta, swa_stream_t stream) {
+    if (bad_theta(theta)) return SWA_ERR_INVALID_ARG;
+    const swa::RopeTable tab = make_rope_table(theta, D);
+    return append_impl(k_new, v_new, k_cache, v_cache, pos, B, T, Hkv, D, W, &tab,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_prefill_rope(const void *q, const void *k, const void *v, void *out, int B, int N,
+                              int Hq, int Hkv, int D, int W, int window_mode, float scale,
+                              float theta, swa_stream_t stream) {
+    if (bad_theta(theta)) return SWA_ERR_INVALID_ARG;
+    const swa::RopeTable tab = make_rope_table(theta, D);
+    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, window_mode, scale, &tab,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_prefill_chunk_rope(const void *q, const void *k, const void *v, void *k_cache,
+                                    void *v_cache, const int32_t *start_pos, void *out, int B,
+                                    int C, int Hq, int Hkv, int D, int W, float scale, float theta,
+                                    swa_stream_t stream) {
+    if (bad_theta(theta)) return SWA_ERR_INVALID_ARG;
+    const swa::RopeTable tab = make_rope_table(theta, D);
+    return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, C, Hq, Hkv, D, W, scale,
+                              &tab, reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_decode_rope(const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
+                             float scale, float theta, void *workspace, size_t workspace_bytes,
+                             swa_stream_t stream) {
+    if (bad_theta(theta)) return SWA_ERR_INVALID_ARG;
+    const swa::RopeTable tab = make_rope_table(theta, D);
+    return decode_impl(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale, workspace,
+                       workspace_bytes, &tab, reinterpret_cast<cudaStream_t>(stream));
 }
 
 swa_status_t swa_get_device_status(swa_stream_t stream) {

@@ -62,5 +62,10 @@ def test_gpu_stack_reach(W, L, mode, span):
     torch.cuda.synchronize()
     diff = (a.float() - b.float()).abs().amax(dim=(0, 2, 3)).cpu().numpy()
     changed = np.nonzero(diff > 0)[0].tolist()
-    assert changed and changed[0] == j and changed[-1] == j + span, (changed[:3], changed[-3:])
+    # nothing outside the reach moves, bit for bit; inside it the change shows
+    # up to the last window (at the exact edge the influence passes through one
+    # key of weight ~1/W per layer and can round away in bf16; the exact edge
+    # is pinned in fp64 by the oracle test above)
+    assert changed and changed[0] == j, changed[:3]
     assert all(diff[i] == 0 for i in range(N) if i < j or i > j + span)
+    assert changed[-1] > j + span - W, (changed[-1], j + span)
