@@ -170,6 +170,33 @@ swa_status_t swa_decode_noalloc(const void *q, const void *k_cache, const void *
                                 int W, float scale, swa_stream_t stream);
 
 /*
+ * Variable-length batches in one launch (serving flow of pre-fill chunks and
+ * decode tokens mixed, section 4.1 and 4.3 of the manon006 review).  The
+ * sequences are packed: q/out [total, Hq, D], k/v [total, Hkv, D] with
+ * sequence b in rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (cu_seqlens: int32
+ * [B+1] device array, cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] =
+ * total; empty sequences allowed).  B <= 256.  Malformed offsets are recorded
+ * as SWA_ERR_INVALID_ARG in the device status word.
+ */
+
+/* swa_prefill_varlen -- one-shot prefill of each sequence (positions 0..n_b-1). */
+swa_status_t swa_prefill_varlen(const void *q, const void *k, const void *v, void *out,
+                                const int32_t *cu_seqlens, int B, int total, int Hq, int Hkv, int D,
+                                int W, int window_mode, float scale, swa_stream_t stream);
+
+/* swa_prefill_chunk_varlen -- one pre-fill chunk per sequence through its
+ * rolling buffer (k_cache, v_cache [B, W, Hkv, D]), sequence b starting at
+ * position start_pos[b].  A sequence of length 1 is a decode step (append,
+ * then attend), so pre-fill chunks and decode tokens share one launch.  Any
+ * length is accepted: a sequence longer than W leaves its last W positions in
+ * the buffer.  Attend first, then write. */
+swa_status_t swa_prefill_chunk_varlen(const void *q, const void *k, const void *v, void *k_cache,
+                                      void *v_cache, const int32_t *start_pos,
+                                      const int32_t *cu_seqlens, void *out, int B, int total,
+                                      int Hq, int Hkv, int D, int W, float scale,
+                                      swa_stream_t stream);
+
+/*
  * Rotary position embedding (RoPE).  The pages give only its base, theta =
  * 10000, in the Table 1 line of "Methods" of the "Mistral 7B -- Sliding
  * Window Attention" summary.  Adopted convention (the original RoFormer

@@ -88,6 +88,10 @@ def lib() -> ctypes.CDLL:
             for fn in (L.swa_rope, L.swa_cache_append_rope, L.swa_prefill_rope, L.swa_prefill_chunk_rope,
                        L.swa_decode_rope):
                 fn.restype = ctypes.c_int
+            L.swa_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, st]
+            L.swa_prefill_chunk_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, st]
+            L.swa_prefill_varlen.restype = ctypes.c_int
+            L.swa_prefill_chunk_varlen.restype = ctypes.c_int
             L.swa_decode_workspace_size.argtypes = [i, i, i, i, i]
             L.swa_decode_workspace_size.restype = ctypes.c_size_t
             L.swa_get_device_status.argtypes = [st]
@@ -257,3 +261,38 @@ def swa_selftest_exp2(x, stream=None):
 
 def swa_selftest_wait_timeout(stream=None) -> None:
     _check(lib().swa_selftest_wait_timeout(_stream_handle(stream)), "swa_selftest_wait_timeout")
+
+
+def swa_prefill_varlen(q, k, v, cu_seqlens, W: int, scale: float, out=None,
+                       window_mode: int = SWA_WINDOW_EXCL_LEFT, stream=None):
+    """One-shot prefill of a packed variable-length batch.  q [total,Hq,D],
+    k/v [total,Hkv,D] bf16; cu_seqlens int32 CUDA [B+1]."""
+    import torch
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().swa_prefill_varlen(_bf16(q, "q"), _bf16(k, "k", (total, Hkv, D)), _bf16(v, "v", (total, Hkv, D)),
+                                    _bf16(out, "out", (total, Hq, D)), _i32(cu_seqlens, "cu_seqlens", B + 1),
+                                    B, total, Hq, Hkv, D, int(W), int(window_mode), float(scale),
+                                    _stream_handle(stream)), "swa_prefill_varlen")
+    return out
+
+
+def swa_prefill_chunk_varlen(q, k, v, k_cache, v_cache, start_pos, cu_seqlens, W: int, scale: float,
+                             out=None, stream=None):
+    """One chunk per sequence of a packed batch through the rolling buffers
+    [B,W,Hkv,D]; a length-1 sequence is a decode step.  Updates the caches."""
+    import torch
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().swa_prefill_chunk_varlen(
+        _bf16(q, "q"), _bf16(k, "k", (total, Hkv, D)), _bf16(v, "v", (total, Hkv, D)),
+        _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _i32(start_pos, "start_pos", B), _i32(cu_seqlens, "cu_seqlens", B + 1), _bf16(out, "out", (total, Hq, D)),
+        B, total, Hq, Hkv, D, int(W), float(scale), _stream_handle(stream)), "swa_prefill_chunk_varlen")
+    return out

@@ -474,6 +474,41 @@ __global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *
 
 namespace swa {
 
+// Rolling-buffer write for a packed variable-length batch: k_new/v_new
+// [total, Hkv, D]; row r belongs to the sequence b with cu[b] <= r < cu[b+1]
+// and has position start_pos[b] + (r - cu[b]).  A sequence longer than W
+// writes only its last W rows (the earlier ones would be overwritten), so no
+// two rows of one call share a slot.
+__global__ void swa_append_varlen_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                                         uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                                         const int32_t *__restrict__ start_pos,
+                                         const int32_t *__restrict__ cu, int B, int total, int W,
+                                         int row_vec) {
+    const long long n = (long long)total * row_vec;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int c = (int)(i % row_vec);
+        const int r = (int)(i / row_vec);
+        int lo = 0, hi = B - 1;                       // last b with cu[b] <= r
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(cu + mid) <= r) lo = mid; else hi = mid - 1;
+        }
+        const int c0 = __ldg(cu + lo), c1 = __ldg(cu + lo + 1);
+        const int s0 = __ldg(start_pos + lo);
+        if (r < c0 || r >= c1 || s0 < 0) {            // malformed offsets or position
+            record_status(kStatusInvalid);
+            continue;
+        }
+        const int t = r - c0;
+        if (t < (c1 - c0) - W) continue;              // overwritten later in this call
+        const int slot = (int)(((long long)s0 + t) % W);
+        const size_t dst = ((size_t)lo * W + slot) * row_vec + c;
+        k_cache[dst] = __ldg(k_new + i);
+        v_cache[dst] = __ldg(v_new + i);
+    }
+}
+
 // In-place rotary embedding of x [B, T, H, D] (bf16), row (b, t) at position
 // pos[b] + t; 16-byte words of four adjacent pairs, grid-stride.
 __global__ void swa_rope_kernel(uint4 *__restrict__ x, const int32_t *__restrict__ pos, int B, int T,

@@ -55,7 +55,12 @@ struct PrefillParams {
     __nv_bfloat16 *out;        // [B, Nq, Hq, D]
     int rope;                  // 1: rotate each Q tile in shared memory after its load
     RopeTable rope_freq;       // theta^(-2i/D), i < D/2
+    // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
+    // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
+    const int32_t *cu_seqlens;
 };
+
+constexpr int kMaxVarlenSeqs = 256;     // sequences per variable-length launch
 
 template <int D>
 struct PrefillCfg {
@@ -73,8 +78,9 @@ struct PrefillCfg {
     // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST],
     // v_empty[VST], s_full[2], p_full[2], o_full[2], drain, p_half[2], q_rot[2]
     static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2 + 2;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag
-    static constexpr int SMEM_BYTES = OFF_MISC + 16;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag, unit count
+    static constexpr int OFF_PRE = OFF_MISC + 16;           // varlen: query-block prefix sums
+    static constexpr int SMEM_BYTES = OFF_PRE + (kMaxVarlenSeqs + 1) * 4;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-byte alignment
     static constexpr int THREADS = 384;
     // which of the 16 column pairs of each 32-column chunk take the polynomial
@@ -104,18 +110,47 @@ struct UnitPlan {
     int nc2, c2;     // cache run 2
     int nm, m0;      // main tiles m0 .. m0+nm-1
     int n;           // total tiles
+    int nq;          // query rows of this sequence (== rows of its main k/v)
+    int row0;        // first packed row of this sequence in q/k/v (varlen), else 0
+    int tb;          // TMA batch coordinate of q/k/v (0 when packed)
+    size_t orow0;    // output row of query row 0 of this sequence
 };
 
-__device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u) {
+// pre: shared-memory prefix sums of query blocks per sequence (varlen only).
+__device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, const int *pre) {
     constexpr int BM = 128, BN = 128;
     UnitPlan P;
-    const int per = p.B * p.Hkv * p.npairs;
-    P.qb = p.nqb - 1 - u / per;          // latest (heaviest) query blocks first
-    int r = u % per;
-    P.pair = r % p.npairs;
-    r /= p.npairs;
-    P.g = r % p.Hkv;
-    P.b = r / p.Hkv;
+    if (p.cu_seqlens) {
+        const int per = p.Hkv * p.npairs;
+        const int qbi = pre[p.B] - 1 - u / per;        // later blocks first
+        int r = u % per;
+        P.pair = r % p.npairs;
+        P.g = r / p.npairs;
+        int lo = 0, hi = p.B - 1;                       // last b with pre[b] <= qbi
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pre[mid] <= qbi) lo = mid; else hi = mid - 1;
+        }
+        P.b = lo;
+        P.qb = qbi - pre[lo];
+        const int c0 = __ldg(p.cu_seqlens + lo);
+        P.nq = max(0, __ldg(p.cu_seqlens + lo + 1) - c0);
+        P.row0 = c0;
+        P.tb = 0;
+        P.orow0 = (size_t)c0;
+    } else {
+        const int per = p.B * p.Hkv * p.npairs;
+        P.qb = p.nqb - 1 - u / per;          // latest (heaviest) query blocks first
+        int r = u % per;
+        P.pair = r % p.npairs;
+        r /= p.npairs;
+        P.g = r % p.Hkv;
+        P.b = r / p.Hkv;
+        P.nq = p.Nq;
+        P.row0 = 0;
+        P.tb = P.b;
+        P.orow0 = (size_t)P.b * p.Nq;
+    }
     P.q0 = P.qb * BM;
     P.act1 = (2 * P.pair + 1) < p.G;
     P.nc1 = P.nc2 = 0;
@@ -124,7 +159,7 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u) {
         P.s0 = 0;
         P.qs = 0;
         const int lo = max(0, P.q0 - p.W + 1);
-        const int hi = min(p.Nk - 1, P.q0 + BM - 1);
+        const int hi = min(P.nq - 1, P.q0 + BM - 1);
         P.m0 = lo / BN;
         P.nm = hi / BN - P.m0 + 1;
     } else {
@@ -154,9 +189,10 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u) {
                 }
             }
         }
-        const int hi = min(p.Nk - 1, P.q0 + BM - 1);
-        P.m0 = 0;
-        P.nm = hi / BN + 1;
+        const int lo = max(0, P.q0 - p.W + 1);          // chunks longer than W
+        const int hi = min(P.nq - 1, P.q0 + BM - 1);
+        P.m0 = lo / BN;
+        P.nm = hi / BN - P.m0 + 1;
     }
     P.n = P.nc1 + P.nc2 + P.nm;
     return P;
@@ -178,7 +214,7 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPl
         const int tile = (j < P.nc1) ? (P.c1 + j) : (P.c2 + (j - P.nc1));
         const int k0 = tile * BN;
         t.row0 = k0;
-        const int t_last = min(P.q0 + BM - 1, p.Nq - 1);
+        const int t_last = min(P.q0 + BM - 1, P.nq - 1);
         const bool has_qs = (k0 <= P.qs) && (P.qs < k0 + BN);
         const int max_age = (k0 + BN - 1 < P.qs) ? (P.qs - k0) : (p.W - (k0 - P.qs));
         const bool clean = !has_qs && (k0 + BN <= p.W) && (max_age < p.W - t_last) &&
@@ -188,7 +224,7 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPl
         t.cache = 0;
         const int k0 = (P.m0 + (j - P.nc1 - P.nc2)) * BN;
         t.row0 = k0;
-        const bool clean = (k0 + BN - 1 <= P.q0) && (k0 > P.q0 + BM - 1 - p.W) && (k0 + BN <= p.Nk);
+        const bool clean = (k0 + BN - 1 <= P.q0) && (k0 > P.q0 + BM - 1 - p.W) && (k0 + BN <= P.nq);
         t.masked = !clean;
     }
     return t;
@@ -243,6 +279,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t bar_q_rot = bar_p_half + 16;               // + 8*t (RoPE on Q done)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::OFF_MISC + 4);
+    int *unit_count = reinterpret_cast<int *>(smem + Cfg::OFF_MISC + 8);
+    int *pre = reinterpret_cast<int *>(smem + Cfg::OFF_PRE);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -271,6 +309,21 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(bar_q_rot + 8, 4);
         *abort_flag = 0;
         mbar_init_fence();
+        if (p.cu_seqlens) {
+            // query blocks per sequence, prefix-summed (empty or malformed
+            // sequences count as empty; malformed ones are recorded)
+            int acc = 0;
+            for (int b = 0; b < p.B; ++b) {
+                pre[b] = acc;
+                const int n = __ldg(p.cu_seqlens + b + 1) - __ldg(p.cu_seqlens + b);
+                if (n < 0) record_status(kStatusInvalid);
+                acc += (max(n, 0) + 127) / 128;
+            }
+            pre[p.B] = acc;
+            *unit_count = acc * p.Hkv * p.npairs;
+        } else {
+            *unit_count = p.num_units;
+        }
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tm_q);
@@ -289,6 +342,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int num_units = *unit_count;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -297,15 +351,15 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             uint32_t k_cnt[KST] = {}, v_cnt[VST] = {};
             uint32_t q_cnt = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++uc) {
-                const UnitPlan P = plan_unit(p, u);
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++uc) {
+                const UnitPlan P = plan_unit(p, u, pre);
                 const int nact = 1 + P.act1;
                 if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
                 mbar_arrive_expect_tx(bar_q_full, nact * TB);
                 for (int t = 0; t < nact; ++t) {
                     const int h = P.g * p.G + 2 * P.pair + t;
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, P.q0, P.b);
+                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, P.row0 + P.q0, P.tb);
                 }
                 ++q_cnt;
                 for (int j = 0; j < P.n; ++j) {
@@ -315,15 +369,17 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t ks = kc % KST, kph = (kc / KST) & 1;
                     if (!mbar_wait_bounded(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, limit)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar_k_full + 8 * ks, TB);
+                    // cache tiles: [B, W] slots of sequence b; main tiles: rows of this sequence
+                    const int krow = T.cache ? T.row0 : P.row0 + T.row0, kb = T.cache ? P.b : P.tb;
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_4d(sK + ks * TB + r * RB, mk, bar_k_full + 8 * ks, r * 64, P.g, T.row0, P.b);
+                        tma_load_4d(sK + ks * TB + r * RB, mk, bar_k_full + 8 * ks, r * 64, P.g, krow, kb);
                     ++k_cnt[ks];
                     ++kc;
                     const uint32_t vs = vc % VST, vph = (vc / VST) & 1;
                     if (!mbar_wait_bounded(bar_v_empty + 8 * vs, vph ^ 1, abort_flag, limit)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar_v_full + 8 * vs, TB);
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_4d(sV + vs * TB + r * RB, mv, bar_v_full + 8 * vs, r * 64, P.g, T.row0, P.b);
+                        tma_load_4d(sV + vs * TB + r * RB, mv, bar_v_full + 8 * vs, r * 64, P.g, krow, kb);
                     ++v_cnt[vs];
                     ++vc;
                 }
@@ -352,8 +408,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             uint32_t pc[2] = {0, 0};
             uint32_t qr1 = 0;                      // units with a second query head
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++uc) {
-                const UnitPlan P = plan_unit(p, u);
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++uc) {
+                const UnitPlan P = plan_unit(p, u, pre);
                 const int n = P.n;
                 if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
                 if (p.rope) {       // the softmax warpgroups rotate Q in place first
@@ -473,8 +529,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float sl2 = p.scale_log2;
         uint32_t sc = 0, oc = 0, qc = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++qc) {
-            const UnitPlan P = plan_unit(p, u);
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++qc) {
+            const UnitPlan P = plan_unit(p, u, pre);
             if (t == 1 && !P.act1) continue;
             const int i_rel = P.q0 + row;                  // query row in the q tensor
             if (p.rope) {
@@ -614,9 +670,9 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             ++oc;
             tc_fence_after();
             const int h = P.g * p.G + 2 * P.pair + t;
-            const bool valid_row = i_rel < p.Nq;
+            const bool valid_row = i_rel < P.nq;
             const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-            __nv_bfloat16 *orow = p.out + (((size_t)P.b * p.Nq + i_rel) * p.Hq + h) * D;
+            __nv_bfloat16 *orow = p.out + ((P.orow0 + i_rel) * p.Hq + h) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];

@@ -246,9 +246,10 @@ swa::RopeTable make_rope_table(float theta, int D) {
     return t;
 }
 
+// cu_seqlens non-null: variable-length batch, tensors packed [N = total rows, H, D].
 swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out, int B, int N,
                           int Hq, int Hkv, int D, int W, int window_mode, float scale,
-                          const swa::RopeTable *rope, cudaStream_t s) {
+                          const swa::RopeTable *rope, const int32_t *cu_seqlens, cudaStream_t s) {
     if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
     if (B < 1 || N < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
@@ -258,16 +259,21 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     long long Weff = (long long)W + (window_mode == SWA_WINDOW_INCL_LEFT ? 1 : 0);
     if (Weff > N) Weff = N;                       // the window never reaches before position 0
     const int G = Hq / Hkv;
+    if (cu_seqlens && (B > swa::kMaxVarlenSeqs || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
+        return B > swa::kMaxVarlenSeqs ? SWA_ERR_UNSUPPORTED : SWA_ERR_INVALID_ARG;
     const long long nqb = (N + 127) / 128;
-    const long long units = (long long)B * Hkv * ((G + 1) / 2) * nqb;
+    // varlen: an upper bound (the kernel counts the real units from cu_seqlens)
+    const long long units = cu_seqlens ? (long long)Hkv * ((G + 1) / 2) * (nqb + B)
+                                       : (long long)B * Hkv * ((G + 1) / 2) * nqb;
     if (units > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
     DeviceInfo *dev = nullptr;
     if (swa_status_t e = device_info(&dev)) return e;
 
+    const int mb = cu_seqlens ? 1 : B;              // packed tensors have one batch row
     CUtensorMap mq, mk, mv;
-    if (swa_status_t e = make_operand_map(&mq, q, D, Hq, N, B)) return e;
-    if (swa_status_t e = make_operand_map(&mk, k, D, Hkv, N, B)) return e;
-    if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, N, B)) return e;
+    if (swa_status_t e = make_operand_map(&mq, q, D, Hq, N, mb)) return e;
+    if (swa_status_t e = make_operand_map(&mk, k, D, Hkv, N, mb)) return e;
+    if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, N, mb)) return e;
 
     swa::PrefillParams p{};
     p.B = B;
@@ -286,31 +292,41 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.rope = rope ? 1 : 0;
     if (rope) p.rope_freq = *rope;
+    p.cu_seqlens = cu_seqlens;
     return D == 128 ? launch_prefill<128>(mq, mk, mv, mk, mv, p, dev->sms, s)
                     : launch_prefill<64>(mq, mk, mv, mk, mv, p, dev->sms, s);
 }
 
+// cu_seqlens non-null: variable-length batch; q/k/v/out packed [C = total rows,
+// H, D], sequence b is rows cu[b]..cu[b+1]-1 (any length; one longer than W
+// leaves its last W positions in the buffer).
 swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, void *k_cache,
                                 void *v_cache, const int32_t *start_pos, void *out, int B, int C,
                                 int Hq, int Hkv, int D, int W, float scale,
-                                const swa::RopeTable *rope, cudaStream_t s) {
+                                const swa::RopeTable *rope, const int32_t *cu_seqlens,
+                                cudaStream_t s) {
     if (!q || !k || !v || !k_cache || !v_cache || !start_pos || !out) return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
         !aligned16(v_cache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
         return SWA_ERR_INVALID_ARG;
-    if (B < 1 || C < 1 || W < 1 || C > W || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
+    if (!cu_seqlens && C > W) return SWA_ERR_INVALID_ARG;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return SWA_ERR_INVALID_ARG;
+    if (cu_seqlens && B > swa::kMaxVarlenSeqs) return SWA_ERR_UNSUPPORTED;
     if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
     const int G = Hq / Hkv;
     const long long nqb = (C + 127) / 128;
-    const long long units = (long long)B * Hkv * ((G + 1) / 2) * nqb;
+    const long long units = cu_seqlens ? (long long)Hkv * ((G + 1) / 2) * (nqb + B)
+                                       : (long long)B * Hkv * ((G + 1) / 2) * nqb;
     if (units > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
     DeviceInfo *dev = nullptr;
     if (swa_status_t e = device_info(&dev)) return e;
 
+    const int mb = cu_seqlens ? 1 : B;
     CUtensorMap mq, mk, mv, mkc, mvc;
-    if (swa_status_t e = make_operand_map(&mq, q, D, Hq, C, B)) return e;
-    if (swa_status_t e = make_operand_map(&mk, k, D, Hkv, C, B)) return e;
-    if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, C, B)) return e;
+    if (swa_status_t e = make_operand_map(&mq, q, D, Hq, C, mb)) return e;
+    if (swa_status_t e = make_operand_map(&mk, k, D, Hkv, C, mb)) return e;
+    if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, C, mb)) return e;
     if (swa_status_t e = make_operand_map(&mkc, k_cache, D, Hkv, W, B)) return e;
     if (swa_status_t e = make_operand_map(&mvc, v_cache, D, Hkv, W, B)) return e;
 
@@ -331,11 +347,21 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.rope = rope ? 1 : 0;
     if (rope) p.rope_freq = *rope;
+    p.cu_seqlens = cu_seqlens;
     swa_status_t e = D == 128 ? launch_prefill<128>(mq, mk, mv, mkc, mvc, p, dev->sms, s)
                               : launch_prefill<64>(mq, mk, mv, mkc, mvc, p, dev->sms, s);
     if (e) return e;
     // attend first, then write the chunk (its keys already rotated) into the buffer
-    return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, nullptr, s);
+    if (!cu_seqlens)
+        return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, nullptr, s);
+    const int row_vec = Hkv * D * 2 / 16;
+    long long blocks = ((long long)C * row_vec + 255) / 256;
+    if (blocks > (long long)dev->sms * 8) blocks = (long long)dev->sms * 8;
+    swa::swa_append_varlen_kernel<<<(int)blocks, 256, 0, s>>>(
+        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_cache),
+        static_cast<uint4 *>(v_cache), start_pos, cu_seqlens, B, C, W, row_vec);
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
 }
 
 swa_status_t append_impl(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
@@ -403,7 +429,7 @@ extern "C" {
 swa_status_t swa_prefill(const void *q, const void *k, const void *v, void *out, int B, int N,
                          int Hq, int Hkv, int D, int W, int window_mode, float scale,
                          swa_stream_t stream) {
-    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, window_mode, scale, nullptr,
+    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, window_mode, scale, nullptr, nullptr,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -411,7 +437,7 @@ swa_status_t swa_prefill_chunk(const void *q, const void *k, const void *v, void
                                void *v_cache, const int32_t *start_pos, void *out, int B, int C,
                                int Hq, int Hkv, int D, int W, float scale, swa_stream_t stream) {
     return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, C, Hq, Hkv, D, W, scale,
-                              nullptr, reinterpret_cast<cudaStream_t>(stream));
+                              nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 swa_status_t swa_cache_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
@@ -476,7 +502,7 @@ swa_status_t swa_prefill_rope(const void *q, const void *k, const void *v, void 
                               float theta, swa_stream_t stream) {
     if (bad_theta(theta)) return SWA_ERR_INVALID_ARG;
     const swa::RopeTable tab = make_rope_table(theta, D);
-    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, window_mode, scale, &tab,
+    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, window_mode, scale, &tab, nullptr,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -487,7 +513,7 @@ swa_status_t swa_prefill_chunk_rope(const void *q, const void *k, const void *v,
     if (bad_theta(theta)) return SWA_ERR_INVALID_ARG;
     const swa::RopeTable tab = make_rope_table(theta, D);
     return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, C, Hq, Hkv, D, W, scale,
-                              &tab, reinterpret_cast<cudaStream_t>(stream));
+                              &tab, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 swa_status_t swa_decode_rope(const void *q, const void *k_cache, const void *v_cache,
@@ -498,6 +524,24 @@ swa_status_t swa_decode_rope(const void *q, const void *k_cache, const void *v_c
     const swa::RopeTable tab = make_rope_table(theta, D);
     return decode_impl(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale, workspace,
                        workspace_bytes, &tab, reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_prefill_varlen(const void *q, const void *k, const void *v, void *out,
+                                const int32_t *cu_seqlens, int B, int total, int Hq, int Hkv, int D,
+                                int W, int window_mode, float scale, swa_stream_t stream) {
+    if (!cu_seqlens) return SWA_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, out, B, total, Hq, Hkv, D, W, window_mode, scale, nullptr, cu_seqlens,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_prefill_chunk_varlen(const void *q, const void *k, const void *v, void *k_cache,
+                                      void *v_cache, const int32_t *start_pos,
+                                      const int32_t *cu_seqlens, void *out, int B, int total,
+                                      int Hq, int Hkv, int D, int W, float scale,
+                                      swa_stream_t stream) {
+    if (!cu_seqlens) return SWA_ERR_INVALID_ARG;
+    return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, total, Hq, Hkv, D, W, scale,
+                              nullptr, cu_seqlens, reinterpret_cast<cudaStream_t>(stream));
 }
 
 swa_status_t swa_get_device_status(swa_stream_t stream) {
