@@ -56,6 +56,11 @@ def _load():
             lib.oracle_swa_decode.argtypes = [dp, dp, dp, ip, ip, dp, i, i, i, i, i, d, i]
             lib.oracle_rope.argtypes = [dp, ip, i, i, i, i, d]
             lib.oracle_rope.restype = ctypes.c_int
+            lib.oracle_swa_prefill_sinks.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, i, d, lp, ctypes.c_int64]
+            lib.oracle_sink_append.argtypes = [vp, vp, vp, vp, ip, i, i, i, i, i, i]
+            lib.oracle_swa_decode_sinks.argtypes = [dp, dp, dp, ip, dp, dp, ip, dp, i, i, i, i, i, i, d]
+            for f in (lib.oracle_swa_prefill_sinks, lib.oracle_sink_append, lib.oracle_swa_decode_sinks):
+                f.restype = ctypes.c_int
             for f in (lib.oracle_swa_prefill, lib.oracle_cache_append, lib.oracle_slot_positions,
                       lib.oracle_swa_chunk, lib.oracle_swa_decode):
                 f.restype = ctypes.c_int
@@ -196,3 +201,53 @@ def rope(x, pos, theta: float = 10000.0) -> np.ndarray:
     if rc != 0:
         raise ValueError("oracle_rope: bad arguments")
     return y
+
+
+def swa_prefill_sinks(q, k, v, W: int, S: int, scale: float, rows=None) -> np.ndarray:
+    """One-shot SWA with S attention-sink positions: query i sees its window
+    (i-W, i] and positions j < S (j <= i).  Shapes as swa_prefill."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if rows is None:
+        out = np.empty((B, N, Hq, D), np.float64)
+        rp, nr = None, 0
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        out = np.empty((B, r.size, Hq, D), np.float64)
+        rp, nr = r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), r.size
+    rc = _load().oracle_swa_prefill_sinks(_dp(q), _dp(k), _dp(v), _dp(out), B, N, Hq, Hkv, D,
+                                          int(W), int(S), float(scale), rp, nr)
+    if rc != 0:
+        raise ValueError("oracle_swa_prefill_sinks: bad arguments")
+    return out
+
+
+def sink_append(k_sink: np.ndarray, v_sink: np.ndarray, k_new, v_new, pos) -> None:
+    """In place: new tokens at positions p < S also go to sink slot p.
+    k_sink, v_sink: [B, S, Hkv, D]; k_new, v_new: [B, T, Hkv, D] (same dtype)."""
+    B, S, Hkv, D = k_sink.shape
+    T = k_new.shape[1]
+    kn = np.ascontiguousarray(k_new, dtype=k_sink.dtype)
+    vn = np.ascontiguousarray(v_new, dtype=k_sink.dtype)
+    rc = _load().oracle_sink_append(k_sink.ctypes.data, v_sink.ctypes.data, kn.ctypes.data, vn.ctypes.data,
+                                    _ip(_i32(pos)), B, T, Hkv, D, S, k_sink.dtype.itemsize)
+    if rc != 0:
+        raise ValueError("oracle_sink_append: bad arguments")
+
+
+def swa_decode_sinks(q, k_cache, v_cache, slot_pos, k_sink, v_sink, pos, W: int, scale: float) -> np.ndarray:
+    """Decode with sinks: window keys from the rolling buffer, sink positions
+    that left the window from the sink buffer [B, S, Hkv, D]."""
+    q = _f64(q)
+    kc, vc, ks, vs = _f64(k_cache), _f64(v_cache), _f64(k_sink), _f64(v_sink)
+    sp, p = _i32(slot_pos), _i32(pos)
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    S = ks.shape[1]
+    out = np.empty((B, Hq, D), np.float64)
+    rc = _load().oracle_swa_decode_sinks(_dp(q), _dp(kc), _dp(vc), _ip(sp), _dp(ks), _dp(vs), _ip(p), _dp(out),
+                                         B, Hq, Hkv, D, int(W), int(S), float(scale))
+    if rc != 0:
+        raise ValueError("oracle_swa_decode_sinks: bad arguments")
+    return out

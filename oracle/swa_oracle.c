@@ -301,3 +301,124 @@ int oracle_swa_decode(const double *q, const double *k_cache,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Attention sinks ([P3] aionda.blog "LLM 추론용 SWA ...", sections "왜 단순
+ * sliding window만으로는 부족한가" and "추론 레이어 SWA가 주는 실용성": keep
+ * the key/values of the first few tokens -- four suffice -- besides the
+ * recent window; the middle is dropped).  Adopted reading: query i sees the
+ * keys of its window (i-W < j <= i) and, in addition, positions j < S
+ * (j <= i), each key once.
+ * ---------------------------------------------------------------------- */
+
+/* One-shot prefill with S sink positions.  Same layout as
+ * oracle_swa_prefill. */
+int oracle_swa_prefill_sinks(const double *q, const double *k, const double *v,
+                             double *out, int B, int N, int Hq, int Hkv, int D,
+                             int W, int S, double scale, const int64_t *rows,
+                             int64_t nrows)
+{
+    if (B < 1 || N < 1 || Hq < 1 || Hkv < 1 || D < 1 || W < 1 || S < 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    const int G = Hq / Hkv;
+    const int64_t nr = rows ? nrows : N;
+    const int64_t total = (int64_t)B * nr * Hq;
+    int bad = 0;
+#pragma omp parallel
+    {
+        const double **kr = malloc(sizeof(double *) * (size_t)N);
+        const double **vr = malloc(sizeof(double *) * (size_t)N);
+        double *sc = malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < total; ++r) {
+            const int h = (int)(r % Hq);
+            const int64_t ri = (r / Hq) % nr;
+            const int b = (int)(r / ((int64_t)Hq * nr));
+            const long i = rows ? (long)rows[ri] : (long)ri;
+            if (i < 0 || i >= N) { bad = 1; continue; }
+            const int g = h / G;
+            long nk = 0;
+            for (long j = 0; j <= i; ++j) {
+                if (!(in_window(i, j, W, ORACLE_WINDOW_EXCL_LEFT) || j < S)) continue;
+                kr[nk] = k + (((size_t)b * N + j) * Hkv + g) * D;
+                vr[nk] = v + (((size_t)b * N + j) * Hkv + g) * D;
+                ++nk;
+            }
+            const double *qr = q + (((size_t)b * N + i) * Hq + h) * D;
+            double *o = out + (((size_t)b * nr + ri) * Hq + h) * D;
+            attend_row(qr, kr, vr, nk, D, scale, sc, o);
+        }
+        free(kr); free(vr); free(sc);
+    }
+    return bad ? -1 : 0;
+}
+
+/* Sink buffer write: new tokens whose position p is below S are also stored
+ * at sink slot p.  k_sink, v_sink : [B, S, Hkv, D]; k_new, v_new :
+ * [B, T, Hkv, D] (bytes copied unchanged). */
+int oracle_sink_append(void *k_sink, void *v_sink, const void *k_new,
+                       const void *v_new, const int32_t *pos, int B, int T,
+                       int Hkv, int D, int S, int elem_bytes)
+{
+    if (B < 1 || T < 0 || Hkv < 1 || D < 1 || S < 0 || elem_bytes < 1) return -1;
+    const size_t row = (size_t)Hkv * D * elem_bytes;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            const long p = (long)pos[b] + t;
+            if (p < 0) return -1;
+            if (p >= S) continue;
+            memcpy((char *)k_sink + ((size_t)b * S + p) * row,
+                   (const char *)k_new + ((size_t)b * T + t) * row, row);
+            memcpy((char *)v_sink + ((size_t)b * S + p) * row,
+                   (const char *)v_new + ((size_t)b * T + t) * row, row);
+        }
+    return 0;
+}
+
+/* Decode with sinks: the keys of the window come from the rolling buffer
+ * (recorded positions in (p-W, p]); sink positions j < S that fell out of the
+ * window (j <= p-W) come from the sink buffer, which holds position j at
+ * slot j. */
+int oracle_swa_decode_sinks(const double *q, const double *k_cache,
+                            const double *v_cache, const int32_t *slot_pos,
+                            const double *k_sink, const double *v_sink,
+                            const int32_t *pos, double *out, int B, int Hq,
+                            int Hkv, int D, int W, int S, double scale)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || W < 1 || S < 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    const int G = Hq / Hkv;
+    const int64_t total = (int64_t)B * Hq;
+#pragma omp parallel
+    {
+        const size_t cap = (size_t)W + (size_t)S;
+        const double **kr = malloc(sizeof(double *) * cap);
+        const double **vr = malloc(sizeof(double *) * cap);
+        double *sc = malloc(sizeof(double) * cap);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < total; ++r) {
+            const int h = (int)(r % Hq);
+            const int b = (int)(r / Hq);
+            const int g = h / G;
+            const long p = pos[b];
+            long nk = 0;
+            for (int s = 0; s < W; ++s) {
+                const long ps = slot_pos[(size_t)b * W + s];
+                if (ps < 0 || !in_window(p, ps, W, ORACLE_WINDOW_EXCL_LEFT)) continue;
+                kr[nk] = k_cache + (((size_t)b * W + s) * Hkv + g) * D;
+                vr[nk] = v_cache + (((size_t)b * W + s) * Hkv + g) * D;
+                ++nk;
+            }
+            for (long j = 0; j < S && j <= p - W; ++j) {
+                kr[nk] = k_sink + (((size_t)b * S + j) * Hkv + g) * D;
+                vr[nk] = v_sink + (((size_t)b * S + j) * Hkv + g) * D;
+                ++nk;
+            }
+            const double *qr = q + ((size_t)b * Hq + h) * D;
+            double *o = out + ((size_t)b * Hq + h) * D;
+            attend_row(qr, kr, vr, nk, D, scale, sc, o);
+        }
+        free(kr); free(vr); free(sc);
+    }
+    return 0;
+}

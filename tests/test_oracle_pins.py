@@ -349,3 +349,47 @@ def test_rope_scores_depend_on_relative_position_only(oracle_mod):
     s1 = float(np.sum(oracle_mod.rope(q, [1000]) * oracle_mod.rope(k, [900])))
     s2 = float(np.sum(oracle_mod.rope(q, [1100 + 4096]) * oracle_mod.rope(k, [1000 + 4096])))
     assert abs(s1 - s2) < 1e-8
+
+
+# ---------------------------------------------------------------- attention sinks
+
+def test_sinks_zero_is_plain_window(oracle_mod):
+    B, N, Hq, Hkv, D = 1, 40, 4, 2, 8
+    q, k, v = _rand((B, N, Hq, D), 50), _rand((B, N, Hkv, D), 51), _rand((B, N, Hkv, D), 52)
+    np.testing.assert_array_equal(oracle_mod.swa_prefill_sinks(q, k, v, 7, 0, 0.3),
+                                  oracle_mod.swa_prefill(q, k, v, 7, 0.3))
+
+
+@pytest.mark.parametrize("W,S", [(5, 4), (1, 2), (3, 10), (40, 4)])
+def test_sinks_brute_force(oracle_mod, W, S):
+    """Key set of row i built as a set union: last W positions, plus the first S."""
+    B, N, Hq, Hkv, D = 1, 30, 2, 1, 8
+    q, k, v = _rand((B, N, Hq, D), 53), _rand((B, N, Hkv, D), 54), _rand((B, N, Hkv, D), 55)
+    out = oracle_mod.swa_prefill_sinks(q, k, v, W, S, 0.4)
+    for i in range(N):
+        keys = sorted(set(sorted(range(i + 1))[-W:]) | set(range(min(S, i + 1))))
+        for h in range(Hq):
+            s = np.array([0.4 * float(q[0, i, h] @ k[0, j, 0]) for j in keys])
+            w = np.exp(s - s.max())
+            w /= w.sum()
+            np.testing.assert_allclose(out[0, i, h], sum(wj * v[0, j, 0] for wj, j in zip(w, keys)),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def test_sink_decode_equals_row_of_prefill(oracle_mod):
+    """Streaming decode with a W-slot rolling buffer plus an S-slot sink buffer
+    equals row p of one-shot prefill with sinks, at every step."""
+    B, N, Hq, Hkv, D, W, S = 2, 45, 4, 2, 8, 8, 4
+    q, k, v = _rand((B, N, Hq, D), 56), _rand((B, N, Hkv, D), 57), _rand((B, N, Hkv, D), 58)
+    one = oracle_mod.swa_prefill_sinks(q, k, v, W, S, 0.3)
+    kc, vc = np.zeros((B, W, Hkv, D)), np.zeros((B, W, Hkv, D))
+    ks, vs = np.zeros((B, S, Hkv, D)), np.zeros((B, S, Hkv, D))
+    sp = np.full((B, W), -1, np.int32)
+    for p in range(N):
+        pos = [p] * B
+        oracle_mod.cache_append(kc, vc, sp, k[:, p:p + 1], v[:, p:p + 1], pos)
+        oracle_mod.sink_append(ks, vs, k[:, p:p + 1], v[:, p:p + 1], pos)
+        out = oracle_mod.swa_decode_sinks(q[:, p], kc, vc, sp, ks, vs, pos, W, 0.3)
+        np.testing.assert_allclose(out, one[:, p], rtol=1e-12, atol=1e-13)
+    # the sink buffer holds exactly the first S positions
+    np.testing.assert_array_equal(ks, k[:, :S])
