@@ -197,6 +197,35 @@ swa_status_t swa_prefill_chunk_varlen(const void *q, const void *k, const void *
                                       swa_stream_t stream);
 
 /*
+ * Attention sinks (StreamingLLM; aionda.blog "LLM 추론용 SWA", sections on why
+ * a plain sliding window is not enough and on inference-time SWA: the first
+ * few tokens -- four suffice -- keep their key/values besides the recent
+ * window, the middle is dropped).  Adopted reading: query i attends to its
+ * window (i-W < j <= i) and to positions j < S, each key once.  The sinks
+ * live in their own buffer k_sink, v_sink [B, S, Hkv, D] (position j at slot
+ * j), beside the W-slot rolling buffer.
+ */
+
+/* swa_prefill_sinks -- one-shot prefill with S sink positions (S >= 0). */
+swa_status_t swa_prefill_sinks(const void *q, const void *k, const void *v, void *out, int B, int N,
+                               int Hq, int Hkv, int D, int W, int S, float scale,
+                               swa_stream_t stream);
+
+/* swa_cache_append_sinks -- swa_cache_append that also stores new tokens
+ * with position p < S at sink slot p. */
+swa_status_t swa_cache_append_sinks(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                                    void *k_sink, void *v_sink, const int32_t *pos, int B, int T,
+                                    int Hkv, int D, int W, int S, swa_stream_t stream);
+
+/* swa_decode_sinks -- swa_decode plus the sink positions that have left the
+ * window (j < S, j <= pos-W), read from the sink buffer.  The workspace is
+ * sized by swa_decode_workspace_size(B, Hq, Hkv, D, W + S). */
+swa_status_t swa_decode_sinks(const void *q, const void *k_cache, const void *v_cache,
+                              const void *k_sink, const void *v_sink, const int32_t *pos, void *out,
+                              int B, int Hq, int Hkv, int D, int W, int S, float scale,
+                              void *workspace, size_t workspace_bytes, swa_stream_t stream);
+
+/*
  * Rotary position embedding (RoPE).  The pages give only its base, theta =
  * 10000, in the Table 1 line of "Methods" of the "Mistral 7B -- Sliding
  * Window Attention" summary.  Adopted convention (the original RoFormer

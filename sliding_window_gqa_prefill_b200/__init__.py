@@ -92,6 +92,11 @@ def lib() -> ctypes.CDLL:
             L.swa_prefill_chunk_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, st]
             L.swa_prefill_varlen.restype = ctypes.c_int
             L.swa_prefill_chunk_varlen.restype = ctypes.c_int
+            L.swa_prefill_sinks.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, st]
+            L.swa_cache_append_sinks.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, st]
+            L.swa_decode_sinks.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, st]
+            for fn in (L.swa_prefill_sinks, L.swa_cache_append_sinks, L.swa_decode_sinks):
+                fn.restype = ctypes.c_int
             L.swa_decode_workspace_size.argtypes = [i, i, i, i, i]
             L.swa_decode_workspace_size.restype = ctypes.c_size_t
             L.swa_get_device_status.argtypes = [st]
@@ -295,4 +300,48 @@ def swa_prefill_chunk_varlen(q, k, v, k_cache, v_cache, start_pos, cu_seqlens, W
         _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
         _i32(start_pos, "start_pos", B), _i32(cu_seqlens, "cu_seqlens", B + 1), _bf16(out, "out", (total, Hq, D)),
         B, total, Hq, Hkv, D, int(W), float(scale), _stream_handle(stream)), "swa_prefill_chunk_varlen")
+    return out
+
+
+def swa_prefill_sinks(q, k, v, W: int, S: int, scale: float, out=None, stream=None):
+    """One-shot prefill where positions j < S stay visible beside each window."""
+    import torch
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().swa_prefill_sinks(_bf16(q, "q"), _bf16(k, "k", (B, N, Hkv, D)), _bf16(v, "v", (B, N, Hkv, D)),
+                                   _bf16(out, "out", (B, N, Hq, D)), B, N, Hq, Hkv, D, int(W), int(S), float(scale),
+                                   _stream_handle(stream)), "swa_prefill_sinks")
+    return out
+
+
+def swa_cache_append_sinks(k_new, v_new, k_cache, v_cache, k_sink, v_sink, pos, stream=None) -> None:
+    """Rolling-buffer write that also keeps positions < S in the sink buffers [B,S,Hkv,D]."""
+    B, T, Hkv, D = k_new.shape
+    W, S = k_cache.shape[1], k_sink.shape[1]
+    _check(lib().swa_cache_append_sinks(
+        _bf16(k_new, "k_new"), _bf16(v_new, "v_new", (B, T, Hkv, D)), _bf16(k_cache, "k_cache", (B, W, Hkv, D)),
+        _bf16(v_cache, "v_cache", (B, W, Hkv, D)), _bf16(k_sink, "k_sink", (B, S, Hkv, D)),
+        _bf16(v_sink, "v_sink", (B, S, Hkv, D)), _i32(pos, "pos", B), B, T, Hkv, D, W, S,
+        _stream_handle(stream)), "swa_cache_append_sinks")
+
+
+def swa_decode_sinks(q, k_cache, v_cache, k_sink, v_sink, pos, scale: float, out=None, workspace=None,
+                     stream=None):
+    """Decode over the window plus the sink positions that left it."""
+    import torch
+    B, Hq, D = q.shape
+    W, Hkv = k_cache.shape[1], k_cache.shape[2]
+    S = k_sink.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = swa_decode_workspace_size(B, Hq, Hkv, D, W + S)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().swa_decode_sinks(
+        _bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _bf16(k_sink, "k_sink", (B, S, Hkv, D)), _bf16(v_sink, "v_sink", (B, S, Hkv, D)), _i32(pos, "pos", B),
+        _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, S, float(scale), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream)), "swa_decode_sinks")
     return out

@@ -102,7 +102,8 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                   const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ pos,
                   __nv_bfloat16 *__restrict__ out, float2 *__restrict__ ws_ml,
                   float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2,
-                  int rope, const RopeTable rope_freq) {
+                  int rope, const RopeTable rope_freq, const __nv_bfloat16 *__restrict__ ksink,
+                  const __nv_bfloat16 *__restrict__ vsink, int S) {
     using Cfg = DecodeCfg<D, G>;
     constexpr int LPR = Cfg::LPR, KPR = Cfg::KPR, KI = Cfg::KI, NV = Cfg::NV;
     constexpr int TLEV = Cfg::TLEV, VPL = Cfg::VPL;
@@ -115,7 +116,11 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         if (threadIdx.x == 0 && split == 0 && g == 0) record_status(kStatusInvalid);
         return;
     }
-    const int L = (p >= W - 1) ? W : p + 1;
+    const int Lw = (p >= W - 1) ? W : p + 1;           // keys in the rolling buffer
+    // sink positions that left the window: slots 0 .. ns-1 of the sink buffer,
+    // numbered after the window's keys
+    const int ns = (S > 0 && p >= W) ? min(S, p - W + 1) : 0;
+    const int L = Lw + ns;
     const int begin = split * kDecodeSplit;
     if (begin >= L) return;
     const int end = min(L, begin + kDecodeSplit);
@@ -152,6 +157,8 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const size_t row_stride = (size_t)Hkv * D;     // elements between consecutive slots
     const __nv_bfloat16 *kbase = kc + ((size_t)b * W * Hkv + g) * D + sub * 8;
     const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv + g) * D + sub * 8;
+    const __nv_bfloat16 *ksbase = ns ? ksink + ((size_t)b * S * Hkv + g) * D + sub * 8 : kbase;
+    const __nv_bfloat16 *vsbase = ns ? vsink + ((size_t)b * S * Hkv + g) * D + sub * 8 : vbase;
 
     const int n_iter_total = (end - begin + KI - 1) / KI;
     const int my_iters = (n_iter_total > warp) ? (n_iter_total - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
@@ -165,8 +172,10 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             const int kr = row * KPR + kk;
             const int key = min(begin + it * KI + kr, end - 1);      // clamp: always in bounds
             const uint32_t off = (uint32_t)((kr * D + sub * 8) * 2);
-            cp_async16(st + off, kbase + (size_t)key * row_stride);
-            cp_async16(st + KI * D * 2 + off, vbase + (size_t)key * row_stride);
+            const bool sink = key >= Lw;
+            const size_t rowi = (size_t)(sink ? key - Lw : key) * row_stride;
+            cp_async16(st + off, (sink ? ksbase : kbase) + rowi);
+            cp_async16(st + KI * D * 2 + off, (sink ? vsbase : vbase) + rowi);
         }
     };
 
@@ -389,12 +398,13 @@ template <int D, int G>
 __global__ void __launch_bounds__(1024)
 swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restrict__ ws_ml,
                           const float *__restrict__ ws_o, __nv_bfloat16 *__restrict__ out,
-                          int Hkv, int W, int nsplit_max) {
+                          int Hkv, int W, int nsplit_max, int S) {
     const int g = blockIdx.x, b = blockIdx.y;
     const int Hq = Hkv * G;
     const int p = __ldg(pos + b);
     if (p < 0) return;
-    const int L = (p >= W - 1) ? W : p + 1;
+    const int ns = (S > 0 && p >= W) ? min(S, p - W + 1) : 0;
+    const int L = ((p >= W - 1) ? W : p + 1) + ns;
     const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
     if (nsplit <= 1) return;
     const size_t base = (size_t)(b * Hkv + g) * nsplit_max;
@@ -446,7 +456,8 @@ swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restr
 __global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                                   uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                                   const int32_t *__restrict__ pos, int B, int T, int W,
-                                  int row_vec, int head_vec, int rope, const RopeTable rope_freq) {
+                                  int row_vec, int head_vec, int rope, const RopeTable rope_freq,
+                                  uint4 *__restrict__ k_sink, uint4 *__restrict__ v_sink, int S) {
     // row_vec = Hkv*D*2/16 sixteen-byte vectors per (b, t) row
     const long long total = (long long)B * T * row_vec;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -465,8 +476,14 @@ __global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *
         const size_t dst = ((size_t)b * W + slot) * row_vec + c;
         uint4 kv = __ldg(k_new + i);
         if (rope) kv = rope_rotate8(kv, (c % head_vec) * 4, (double)p, rope_freq);
+        const uint4 vv = __ldg(v_new + i);
         k_cache[dst] = kv;
-        v_cache[dst] = __ldg(v_new + i);
+        v_cache[dst] = vv;
+        if (p < S) {                     // attention sinks: positions below S kept for good
+            const size_t sdst = ((size_t)b * S + p) * row_vec + c;
+            k_sink[sdst] = kv;
+            v_sink[sdst] = vv;
+        }
     }
 }
 

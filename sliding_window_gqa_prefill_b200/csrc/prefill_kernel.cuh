@@ -58,6 +58,9 @@ struct PrefillParams {
     // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
     // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
     const int32_t *cu_seqlens;
+    // attention sinks (one-shot prefill): positions j < sinks stay visible to
+    // every query besides its window
+    int sinks;
 };
 
 constexpr int kMaxVarlenSeqs = 256;     // sequences per variable-length launch
@@ -109,6 +112,7 @@ struct UnitPlan {
     int nc1, c1;     // cache run 1: tiles c1 .. c1+nc1-1
     int nc2, c2;     // cache run 2
     int nm, m0;      // main tiles m0 .. m0+nm-1
+    int sink_tile;   // main tiles 0 .. sink_tile-1 below the band, visited first for the sinks
     int n;           // total tiles
     int nq;          // query rows of this sequence (== rows of its main k/v)
     int row0;        // first packed row of this sequence in q/k/v (varlen), else 0
@@ -162,7 +166,10 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         const int hi = min(P.nq - 1, P.q0 + BM - 1);
         P.m0 = lo / BN;
         P.nm = hi / BN - P.m0 + 1;
+        // sink positions below the band live in the first ceil(S/128) tiles
+        P.sink_tile = min((p.sinks + BN - 1) / BN, P.m0);
     } else {
+        P.sink_tile = 0;
         P.s0 = __ldg(p.start_pos + P.b);
         if (P.s0 < 0) {                       // invalid start: record it, attend as if 0
             record_status(kStatusInvalid);
@@ -194,7 +201,7 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         P.m0 = lo / BN;
         P.nm = hi / BN - P.m0 + 1;
     }
-    P.n = P.nc1 + P.nc2 + P.nm;
+    P.n = P.sink_tile + P.nc1 + P.nc2 + P.nm;
     return P;
 }
 
@@ -209,6 +216,13 @@ struct TileRef {
 __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPlan &P, int j) {
     constexpr int BM = 128, BN = 128;
     TileRef t;
+    if (j < P.sink_tile) {                  // only the sink positions of this tile count
+        t.cache = 0;
+        t.row0 = j * BN;
+        t.masked = 1;
+        return t;
+    }
+    j -= P.sink_tile;
     if (j < P.nc1 + P.nc2) {
         t.cache = 1;
         const int tile = (j < P.nc1) ? (P.c1 + j) : (P.c2 + (j - P.nc1));
@@ -582,7 +596,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                         for (int c = 0; c < BN; ++c) {
                             const int key = T.row0 + c;
-                            if (key > i_rel || key <= i_rel - p.W) s[c] = -INFINITY;
+                            if (key > i_rel || (key <= i_rel - p.W && key >= p.sinks)) s[c] = -INFINITY;
                         }
                     }
                 }

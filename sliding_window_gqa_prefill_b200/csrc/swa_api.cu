@@ -134,7 +134,8 @@ swa_status_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const 
 
 swa_status_t launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
                            const int32_t *pos, int B, int T, int Hkv, int D, int W, int sms,
-                           const swa::RopeTable *rope, cudaStream_t s) {
+                           const swa::RopeTable *rope, cudaStream_t s, void *k_sink = nullptr,
+                           void *v_sink = nullptr, int S = 0) {
     const int row_vec = Hkv * D * 2 / 16;
     const long long total = (long long)B * T * row_vec;
     long long blocks = (total + 255) / 256;
@@ -144,7 +145,8 @@ swa_status_t launch_append(const void *k_new, const void *v_new, void *k_cache, 
     swa::swa_append_kernel<<<(int)blocks, 256, 0, s>>>(
         static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
         static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), pos, B, T, W, row_vec, D / 8,
-        rope ? 1 : 0, rope ? *rope : swa::RopeTable{});
+        rope ? 1 : 0, rope ? *rope : swa::RopeTable{}, static_cast<uint4 *>(k_sink),
+        static_cast<uint4 *>(v_sink), S);
     SWA_CUDA_TRY(cudaGetLastError());
     return SWA_OK;
 }
@@ -154,8 +156,9 @@ int decode_nsplit_max(int W) { return (W + swa::kDecodeSplit - 1) / swa::kDecode
 template <int D, int G>
 swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, const int32_t *pos,
                               void *out, int B, int Hkv, int W, float scale, void *ws,
-                              const swa::RopeTable *rope, cudaStream_t s) {
-    const int nsm = decode_nsplit_max(W);
+                              const swa::RopeTable *rope, cudaStream_t s, const void *ksink,
+                              const void *vsink, int S) {
+    const int nsm = decode_nsplit_max(W + S);
     const size_t o_elems = (size_t)B * Hkv * nsm * G * D;
     float *ws_o = static_cast<float *>(ws);
     float2 *ws_ml = ws ? reinterpret_cast<float2 *>(static_cast<char *>(ws) + ((o_elems * 4 + 255) & ~size_t(255)))
@@ -164,11 +167,12 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
     swa::swa_decode_kernel<D, G><<<grid, swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
         static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
-        Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{});
+        Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{},
+        static_cast<const __nv_bfloat16 *>(ksink), static_cast<const __nv_bfloat16 *>(vsink), S);
     SWA_CUDA_TRY(cudaGetLastError());
     if (nsm > 1) {
         swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), G * D, 0, s>>>(
-            pos, ws_ml, ws_o, static_cast<__nv_bfloat16 *>(out), Hkv, W, nsm);
+            pos, ws_ml, ws_o, static_cast<__nv_bfloat16 *>(out), Hkv, W, nsm, S);
         SWA_CUDA_TRY(cudaGetLastError());
     }
     return SWA_OK;
@@ -177,12 +181,13 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
 template <int D>
 swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *vc,
                              const int32_t *pos, void *out, int B, int Hkv, int W, float scale,
-                             void *ws, const swa::RopeTable *rope, cudaStream_t s) {
+                             void *ws, const swa::RopeTable *rope, cudaStream_t s,
+                             const void *ksink = nullptr, const void *vsink = nullptr, int S = 0) {
     switch (G) {
-        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
-        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
-        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
-        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s);
+        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         default: return SWA_ERR_UNSUPPORTED;
     }
 }
@@ -249,7 +254,8 @@ swa::RopeTable make_rope_table(float theta, int D) {
 // cu_seqlens non-null: variable-length batch, tensors packed [N = total rows, H, D].
 swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out, int B, int N,
                           int Hq, int Hkv, int D, int W, int window_mode, float scale,
-                          const swa::RopeTable *rope, const int32_t *cu_seqlens, cudaStream_t s) {
+                          const swa::RopeTable *rope, const int32_t *cu_seqlens, cudaStream_t s,
+                          int sinks = 0) {
     if (!q || !k || !v || !out) return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_INVALID_ARG;
     if (B < 1 || N < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
@@ -293,6 +299,7 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.rope = rope ? 1 : 0;
     if (rope) p.rope_freq = *rope;
     p.cu_seqlens = cu_seqlens;
+    p.sinks = sinks;
     return D == 128 ? launch_prefill<128>(mq, mk, mv, mk, mv, p, dev->sms, s)
                     : launch_prefill<64>(mq, mk, mv, mk, mv, p, dev->sms, s);
 }
@@ -542,6 +549,53 @@ swa_status_t swa_prefill_chunk_varlen(const void *q, const void *k, const void *
     if (!cu_seqlens) return SWA_ERR_INVALID_ARG;
     return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, total, Hq, Hkv, D, W, scale,
                               nullptr, cu_seqlens, reinterpret_cast<cudaStream_t>(stream));
+}
+
+swa_status_t swa_prefill_sinks(const void *q, const void *k, const void *v, void *out, int B, int N,
+                               int Hq, int Hkv, int D, int W, int S, float scale, swa_stream_t stream) {
+    if (S < 0) return SWA_ERR_INVALID_ARG;
+    return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, SWA_WINDOW_EXCL_LEFT, scale, nullptr, nullptr,
+                        reinterpret_cast<cudaStream_t>(stream), S);
+}
+
+swa_status_t swa_cache_append_sinks(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                                    void *k_sink, void *v_sink, const int32_t *pos, int B, int T,
+                                    int Hkv, int D, int W, int S, swa_stream_t stream) {
+    if (S < 0 || (S > 0 && (!k_sink || !v_sink || !aligned16(k_sink) || !aligned16(v_sink))))
+        return SWA_ERR_INVALID_ARG;
+    if (!k_new || !v_new || !k_cache || !v_cache || !pos) return SWA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return SWA_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || W < 1 || T > W || Hkv < 1) return SWA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+    return launch_append(k_new, v_new, k_cache, v_cache, pos, B, T, Hkv, D, W, dev->sms, nullptr,
+                         reinterpret_cast<cudaStream_t>(stream), k_sink, v_sink, S);
+}
+
+swa_status_t swa_decode_sinks(const void *q, const void *k_cache, const void *v_cache,
+                              const void *k_sink, const void *v_sink, const int32_t *pos, void *out,
+                              int B, int Hq, int Hkv, int D, int W, int S, float scale,
+                              void *workspace, size_t workspace_bytes, swa_stream_t stream) {
+    if (S < 0 || (S > 0 && (!k_sink || !v_sink || !aligned16(k_sink) || !aligned16(v_sink))))
+        return SWA_ERR_INVALID_ARG;
+    if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
+    if ((long long)W + S > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
+    const size_t need = decode_workspace_bytes(B, Hq, Hkv, D, W + S);
+    if (decode_nsplit_max(W + S) > 1) {
+        if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
+    }
+    DeviceInfo *dev = nullptr;
+    if (swa_status_t e = device_info(&dev)) return e;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int G = Hq / Hkv;
+    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, nullptr, s,
+                                           k_sink, v_sink, S)
+                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, nullptr, s,
+                                          k_sink, v_sink, S);
 }
 
 swa_status_t swa_get_device_status(swa_stream_t stream) {
