@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import itertools
 import json
 import os
 import statistics
@@ -372,6 +373,9 @@ def run_native(args):
 
     launches_per_step = 1 + len(c_chunks) * 2 + dw.steps * (2 + (1 if ws_bytes and dw.W > 512 else 0))
 
+    # ---- the widened rows, timed on their own (CUDA events, after the step)
+    extras = measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, max(3, args.steps // 2), world)
+
     result = None
     if rank == 0:
         cpu = None
@@ -447,6 +451,7 @@ def run_native(args):
                         "frac": chunk_tflops / world / peaks["bf16"]},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
+            "extras": extras,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": status,
@@ -458,6 +463,86 @@ def run_native(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return result
+
+
+def _time_ms(fn, iters: int) -> float:
+    """Median CUDA-event time of fn() on the current stream, after one warm-up."""
+    import torch
+    fn()
+    ts = []
+    for _ in range(iters):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, iters, world):
+    """RoPE-fused prefill and decode, attention sinks, and a mixed
+    variable-length launch (pre-fill chunks and decode tokens together), on the
+    headline shapes; each reported with its useful work rate."""
+    import torch
+    theta, S = 10000.0, 4
+    res = {}
+    out = torch.empty_like(q)
+    kr = k.clone()
+    swa.swa_rope(kr, torch.zeros(hp.B, dtype=torch.int32, device=dev), theta)
+    flops = wl.useful_flops(hp.B, hp.N, hp.W, hp.Hq, hp.D)
+    ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill(q, kr, v, hp.W, hp.scale, out=out, rope_theta=theta),
+                                 iters), world)
+    res["prefill_rope_q_fused"] = {"tflops": flops / ms / 1e9, "ms": ms,
+                                   "note": "q rotated in shared memory after its TMA load; k pre-rotated"}
+    sink_pairs = sum(max(0, min(S, i - hp.W + 1)) for i in range(hp.N))   # sink keys outside the window
+    sflops = flops + 4 * hp.B * hp.Hq * hp.D * sink_pairs
+    ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill_sinks(q, k, v, hp.W, S, hp.scale, out=out), iters), world)
+    res["prefill_sinks4"] = {"tflops": sflops / ms / 1e9, "ms": ms}
+    # decode with fused RoPE and with sinks: one step at B=64 (append + decode)
+    kc, vc = dd["k_cache"].to(dev), dd["v_cache"].to(dev)
+    ks = torch.zeros(dw.B, S, dw.Hkv, dw.D, dtype=torch.bfloat16, device=dev)
+    vs = torch.zeros_like(ks)
+    qd = dd["q"][0].to(dev)
+    kn = dd["k_new"][0].to(dev).unsqueeze(1).contiguous()
+    vn = dd["v_new"][0].to(dev).unsqueeze(1).contiguous()
+    pos = dd["pos0"].to(dev)
+    od = torch.empty_like(qd)
+    ws = torch.empty(max(256, swa.swa_decode_workspace_size(dw.B, dw.Hq, dw.Hkv, dw.D, dw.W + S)),
+                     dtype=torch.uint8, device=dev)
+
+    def dec_rope():
+        swa.swa_cache_append(kn, vn, kc, vc, pos, rope_theta=theta)
+        swa.swa_decode(qd, kc, vc, pos, dw.scale, out=od, workspace=ws, rope_theta=theta)
+
+    def dec_sinks():
+        swa.swa_cache_append_sinks(kn, vn, kc, vc, ks, vs, pos)
+        swa.swa_decode_sinks(qd, kc, vc, ks, vs, pos, dw.scale, out=od, workspace=ws)
+
+    for name, fn in (("decode_rope_step", dec_rope), ("decode_sinks4_step", dec_sinks)):
+        ms = max_over_ranks(_time_ms(fn, iters * 4), world)
+        res[name] = {"tokens_per_s": dw.B * world / (ms * 1e-3), "us": ms * 1e3}
+    # mixed launch: 4 sequences pre-fill a 4096-token chunk, 60 decode one token
+    nseq, nchunk, C = 64, 4, 4096
+    lens = [C] * nchunk + [1] * (nseq - nchunk)
+    total = sum(lens)
+    cu = torch.tensor([0] + list(itertools.accumulate(lens)), dtype=torch.int32, device=dev)
+    start = pos[:nseq].clone()
+    qm = wl.random_bf16((total, hp.Hq, hp.D), 7001).to(dev)
+    km = wl.random_bf16((total, hp.Hkv, hp.D), 7002).to(dev)
+    vm = wl.random_bf16((total, hp.Hkv, hp.D), 7003).to(dev)
+    om = torch.empty_like(qm)
+    kcm, vcm = kc[:nseq].contiguous(), vc[:nseq].contiguous()
+    ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill_chunk_varlen(qm, km, vm, kcm, vcm, start, cu, dw.W,
+                                                                       hp.scale, out=om), iters), world)
+    # useful pairs: each chunk row sees min(W, s0 + t + 1) keys; each decode row min(W, s0 + 1)
+    pairs = 0
+    s0 = start.cpu().tolist()
+    for b, n in enumerate(lens):
+        pairs += sum(min(dw.W, s0[b] + t + 1) for t in range(n))
+    res["varlen_mixed_4x4096_plus_60_decode"] = {"tflops": 4 * hp.Hq * hp.D * pairs * world / ms / 1e9,
+                                                 "ms": ms, "tokens": total}
+    return res
 
 
 def run_reference(args):

@@ -96,7 +96,9 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
 // Partial result of one (sequence, kv head, split): per head m (base-2 max),
 // l (sum of 2^(s-m)) and o[D] (sum of 2^(s-m) v).  Layout in the workspace:
 // ml[((b*Hkv + g)*nsplit_max + s)*G + h] = {m, l};  o[...*D + d].
-template <int D, int G>
+// SINKS: keys past the window's come from the sink buffer (attention sinks);
+// compiled out of the plain decode.
+template <int D, int G, bool SINKS>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
 swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kc,
                   const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ pos,
@@ -119,7 +121,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const int Lw = (p >= W - 1) ? W : p + 1;           // keys in the rolling buffer
     // sink positions that left the window: slots 0 .. ns-1 of the sink buffer,
     // numbered after the window's keys
-    const int ns = (S > 0 && p >= W) ? min(S, p - W + 1) : 0;
+    const int ns = (SINKS && S > 0 && p >= W) ? min(S, p - W + 1) : 0;
     const int L = Lw + ns;
     const int begin = split * kDecodeSplit;
     if (begin >= L) return;
@@ -172,10 +174,15 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             const int kr = row * KPR + kk;
             const int key = min(begin + it * KI + kr, end - 1);      // clamp: always in bounds
             const uint32_t off = (uint32_t)((kr * D + sub * 8) * 2);
-            const bool sink = key >= Lw;
-            const size_t rowi = (size_t)(sink ? key - Lw : key) * row_stride;
-            cp_async16(st + off, (sink ? ksbase : kbase) + rowi);
-            cp_async16(st + KI * D * 2 + off, (sink ? vsbase : vbase) + rowi);
+            if (SINKS) {
+                const bool sink = key >= Lw;
+                const size_t rowi = (size_t)(sink ? key - Lw : key) * row_stride;
+                cp_async16(st + off, (sink ? ksbase : kbase) + rowi);
+                cp_async16(st + KI * D * 2 + off, (sink ? vsbase : vbase) + rowi);
+            } else {
+                cp_async16(st + off, kbase + (size_t)key * row_stride);
+                cp_async16(st + KI * D * 2 + off, vbase + (size_t)key * row_stride);
+            }
         }
     };
 

@@ -97,7 +97,10 @@ swa_status_t device_info(DeviceInfo **out) {
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           swa::PrefillCfg<128>::SMEM_ALLOC));
 #define SWA_SET_DECODE_ATTR(DD, GG)                                                           \
-    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG>,                        \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, false>,                 \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                      swa::DecodeCfg<DD, GG>::SMEM_BYTES));                  \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, true>,                  \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,           \
                                       swa::DecodeCfg<DD, GG>::SMEM_BYTES));
         SWA_SET_DECODE_ATTR(64, 1) SWA_SET_DECODE_ATTR(64, 2) SWA_SET_DECODE_ATTR(64, 4)
@@ -164,7 +167,8 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
     float2 *ws_ml = ws ? reinterpret_cast<float2 *>(static_cast<char *>(ws) + ((o_elems * 4 + 255) & ~size_t(255)))
                        : nullptr;
     dim3 grid(nsm, Hkv, B);
-    swa::swa_decode_kernel<D, G><<<grid, swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
+    auto kernel = S > 0 ? swa::swa_decode_kernel<D, G, true> : swa::swa_decode_kernel<D, G, false>;
+    kernel<<<grid, swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
         static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
         Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{},
