@@ -92,8 +92,6 @@ struct PrefillCfg {
     // PV in two halves of 64 keys: the first half starts while the softmax
     // still computes the second half of P
     static constexpr bool kSplitPV = true;
-    // row maximum with three-input max instructions
-    static constexpr bool kMax3 = false;
     // the MMA thread polls its barriers instead of suspending on them
     static constexpr bool kMmaSpin = false;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -601,21 +599,12 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 float mx[8];
-                if constexpr (Cfg::kMax3) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(s[e], s[8 + e]);
+                for (int e = 0; e < 8; ++e) mx[e] = s[e];
 #pragma unroll
-                    for (int c = 16; c < BN; c += 16)
+                for (int c = 8; c < BN; c += 8)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) mx[e] = fmax3f(mx[e], s[c + e], s[c + 8 + e]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) mx[e] = s[e];
-#pragma unroll
-                    for (int c = 8; c < BN; c += 8)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
-                }
+                    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
                 const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                 const float m_tile = mt * sl2;
