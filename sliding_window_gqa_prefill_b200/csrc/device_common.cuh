@@ -345,6 +345,48 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                        __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Rotary embedding frequencies theta^(-2i/D), i < D/2, computed on the host
+// in double precision and passed by value.
+struct RopeTable {
+    double f[64];
+};
+
+// Generic-proxy writes to shared memory become visible to the async proxy
+// (TMA, tensor core) after this fence.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// cos and sin of p * f: the angle is formed and reduced to [-pi, pi] in
+// double precision, then evaluated with the fast single-precision intrinsic
+// (absolute error below 2^-21 on [-pi, pi], far below the bf16 step).
+__device__ __forceinline__ void rope_cos_sin(double p, double f, float &c, float &s) {
+    constexpr double kTwoPi = 6.283185307179586;
+    const double a = p * f;
+    const double r = fma(-rint(a * (1.0 / kTwoPi)), kTwoPi, a);
+    __sincosf((float)r, &s, &c);
+}
+
+// Rotate four adjacent (even, odd) bf16 pairs held in a 16-byte word; pairs
+// i0 .. i0+3 of the row, position p.
+__device__ __forceinline__ uint4 rope_rotate8(uint4 w, int i0, double p, const RopeTable &tab) {
+    uint32_t in[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float c, s;
+        rope_cos_sin(p, tab.f[i0 + e], c, s);
+        const float x0 = __uint_as_float(in[e] << 16), x1 = __uint_as_float(in[e] & 0xFFFF0000u);
+        in[e] = pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+    }
+    return make_uint4(in[0], in[1], in[2], in[3]);
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
