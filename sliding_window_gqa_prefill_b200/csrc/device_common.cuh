@@ -101,6 +101,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Clean-up waits (copies and MMAs this thread already started) have their own
+// bound, independent of the wait limit a caller may have shortened: work in
+// flight completes in microseconds, and the block must not exit before it has.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+
 // Same, for the clean-up path: ignores *abort, only the time limit ends it.
 __device__ __forceinline__ bool mbar_drain_bounded(uint32_t bar, uint32_t parity,
                                                    unsigned long long limit_ns) {

@@ -398,11 +398,11 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             if (!ok) {
                 // let every copy this thread started land before the block exits
-                if (q_cnt) mbar_drain_bounded(bar_q_full, (q_cnt - 1) & 1, limit);
+                if (q_cnt) mbar_drain_bounded(bar_q_full, (q_cnt - 1) & 1, kDrainLimitNs);
                 for (int s = 0; s < KST; ++s)
-                    if (k_cnt[s]) mbar_drain_bounded(bar_k_full + 8 * s, (k_cnt[s] - 1) & 1, limit);
+                    if (k_cnt[s]) mbar_drain_bounded(bar_k_full + 8 * s, (k_cnt[s] - 1) & 1, kDrainLimitNs);
                 for (int s = 0; s < VST; ++s)
-                    if (v_cnt[s]) mbar_drain_bounded(bar_v_full + 8 * s, (v_cnt[s] - 1) & 1, limit);
+                    if (v_cnt[s]) mbar_drain_bounded(bar_v_full + 8 * s, (v_cnt[s] - 1) & 1, kDrainLimitNs);
             }
         }
         __syncwarp();
@@ -526,7 +526,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             if (!ok) {
                 mma_commit(bar_drain);
-                mbar_drain_bounded(bar_drain, 0, limit);
+                mbar_drain_bounded(bar_drain, 0, kDrainLimitNs);
             }
         }
         __syncwarp();
