@@ -20,7 +20,10 @@
 //  * per key: partial dot products for all G heads of the group, reduced
 //    across the D/8 lanes of the row by a transposing butterfly (each level
 //    halves the values a lane holds), so a key x head score costs about one
-//    shuffle.  Online softmax per head in base 2 (scale folded into q).
+//    shuffle.  Online softmax per head in base 2 (scale folded into q); the
+//    exponent offset of a head is raised (exact maximum over the iteration,
+//    rescale of l and o) only when a score exceeds it by more than 2^8, so
+//    most iterations skip the per-iteration maximum entirely.
 //  * warps and splits are merged by log-sum-exp: in shared memory inside a
 //    block, and by swa_decode_combine_kernel across splits.
 #pragma once
@@ -268,39 +271,52 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                 for (int i = 0; i < VPL; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
             }
         }
-        // scores of this iteration to shared memory, [KI][G]; keys past the split masked
+        // keys past the split masked; a score more than 2^8 above the running
+        // offset of its head (always so on the first iteration) makes the warp
+        // take the exact maximum over the iteration and rescale; otherwise the
+        // offset stays (p = 2^(s - offset) <= 2^8, exact after normalisation)
+        bool big = false;
         if (writer) {
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
                 const int idx = vidx0 + i;
-                const int kr = row * KPR + idx / G;
+                const int kr = row * KPR + idx / G, h = idx % G;
                 v[i] = (key_base + kr < end) ? v[i] : -INFINITY;
-                score[kr * G + idx % G] = v[i];
+                float mh = m_run[0];
+#pragma unroll
+                for (int hh = 1; hh < G; ++hh) mh = (h == hh) ? m_run[hh] : mh;
+                big |= v[i] > mh + 8.0f;
             }
         }
-        __syncwarp();
-        float m_new[G];
+        if (__any_sync(0xffffffffu, big)) {
+            if (writer) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) m_new[h] = m_run[h];
+                for (int i = 0; i < VPL; ++i) {
+                    const int idx = vidx0 + i;
+                    score[(row * KPR + idx / G) * G + idx % G] = v[i];
+                }
+            }
+            __syncwarp();
+            float m_new[G];
 #pragma unroll
-        for (int kr = 0; kr < KI; ++kr) {
-            float sv[G];
-            load_g<G>(score + kr * G, sv);
+            for (int h = 0; h < G; ++h) m_new[h] = m_run[h];
 #pragma unroll
-            for (int h = 0; h < G; ++h) m_new[h] = fmaxf(m_new[h], sv[h]);
-        }
-        __syncwarp();                        // every lane has read the scores
-        bool grow = false;
+            for (int kr = 0; kr < KI; ++kr) {
+                float sv[G];
+                load_g<G>(score + kr * G, sv);
 #pragma unroll
-        for (int h = 0; h < G; ++h) grow |= m_new[h] > m_run[h];
-        if (grow) {                          // uniform across the warp
+                for (int h = 0; h < G; ++h) m_new[h] = fmaxf(m_new[h], sv[h]);
+            }
+            __syncwarp();                        // every lane has read the scores
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                const float alpha = ex2_approx(m_run[h] - m_new[h]);   // 0 when m_run = -inf
-                l_run[h] *= alpha;
+                if (m_new[h] > m_run[h]) {       // uniform across the warp
+                    const float alpha = ex2_approx(m_run[h] - m_new[h]);   // 0 when m_run = -inf
+                    l_run[h] *= alpha;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) o2[h][e] = make_float2(o2[h][e].x * alpha, o2[h][e].y * alpha);
-                m_run[h] = m_new[h];
+                    for (int e = 0; e < 4; ++e) o2[h][e] = make_float2(o2[h][e].x * alpha, o2[h][e].y * alpha);
+                    m_run[h] = m_new[h];
+                }
             }
         }
         // one exponential per key x head, by the lane that holds it
