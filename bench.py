@@ -45,6 +45,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
+    ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
+                    help="run a reduced case of one kernel three times for an ncu capture (no timing)")
     return ap.parse_args(argv)
 
 
@@ -58,22 +60,29 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
-def kernel_source_hash() -> str:
+# the sources each kernel is built from (its launch code is in swa_api.cu)
+KERNEL_SOURCES = {
+    "swa_prefill_kernel<128>": ("device_common.cuh", "prefill_kernel.cuh", "swa_api.cu"),
+    "swa_decode_kernel<128,4>": ("device_common.cuh", "decode_kernel.cuh", "swa_api.cu"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in ("device_common.cuh", "prefill_kernel.cuh", "decode_kernel.cuh", "swa_api.cu"):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, "sliding_window_gqa_prefill_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current sources of that kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
@@ -585,8 +594,48 @@ def run_reference(args):
     }
 
 
+def run_ncu_case(case: str) -> None:
+    """Reduced launches for ncu captures, the benchmark's kernels on a fraction
+    of its workload that still exceeds L2: prefill B=1 (half the headline
+    prefill, same per-unit structure), decode B=16 (a quarter of the batch,
+    positions from the same distribution).  Prints the algorithmic bytes per
+    launch so a capture's DRAM traffic can be scaled to the full launch."""
+    import dataclasses
+    import torch
+    import sliding_window_gqa_prefill_b200 as swa
+    from sliding_window_gqa_prefill_b200 import workloads as wl
+    swa.lib()
+    if case == "prefill":
+        w = dataclasses.replace(wl.HEADLINE_PREFILL, B=1)
+        q, k, v = (t.cuda() for t in wl.prefill_inputs(w))
+        for _ in range(3):
+            swa.swa_prefill(q, k, v, w.W, w.scale)
+        alg = (q.numel() + k.numel() + v.numel() + q.numel()) * 2
+        print(f"ncu case prefill {w.name} B=1: algorithmic bytes per launch {alg}, "
+              f"useful FLOPs {wl.useful_flops(w.B, w.N, w.W, w.Hq, w.D)}")
+    else:
+        w = dataclasses.replace(wl.DECODE_B64, B=16, steps=1)
+        d = wl.decode_inputs(w)
+        kc, vc, pos = d["k_cache"].cuda(), d["v_cache"].cuda(), d["pos0"].cuda()
+        q = d["q"][0].cuda().contiguous()
+        ws = torch.empty(swa.swa_decode_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.W), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(3):
+            swa.swa_decode(q, kc, vc, pos, w.scale, workspace=ws)
+        keys = sum(min(int(p) + 1, w.W) for p in d["pos0"])
+        alg = keys * w.Hkv * w.D * 2 * 2 + q.numel() * 2 * 2
+        print(f"ncu case decode B=16 W={w.W}: algorithmic bytes per launch {alg} (K/V rows in the window "
+              f"+ q + out)")
+    torch.cuda.synchronize()
+    if swa.swa_get_device_status() != 0:
+        raise SystemExit("device status not OK")
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.ncu_case:
+        run_ncu_case(args.ncu_case)
+        return
     os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
     if args.impl == "reference":
         res = run_reference(args)
