@@ -408,6 +408,7 @@ def run_native(args):
 
     # ---- the widened rows, timed on their own (CUDA events, after the step)
     extras = measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, max(3, args.steps // 2), world)
+    sweep = measure_sweep(swa, wl, dev, max(3, args.steps // 2), world)
 
     result = None
     if rank == 0:
@@ -485,6 +486,7 @@ def run_native(args):
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "extras": extras,
+            "sweep": sweep,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": status,
@@ -511,6 +513,34 @@ def _time_ms(fn, iters: int) -> float:
         b.synchronize()
         ts.append(a.elapsed_time(b))
     return statistics.median(ts)
+
+
+def measure_sweep(swa, wl, dev, iters, world):
+    """The long-prefill sweep (B=2, 32/8 heads, D=128): N in {4K, 8K, 16K, 32K}
+    x W in {1024, 4096}, plus the dense-causal control W = N; useful TFLOP/s
+    and ms per launch (CUDA events, median).  Inputs are drawn on the device
+    (N(0,1) bf16, 1% of key rows x8), for timing only: the same shapes are
+    checked against the oracle in the tests.  Also the time ratio of dense
+    causal to W=4096 at N=16K, the pages' "about 2x faster at 16K" setting."""
+    import torch
+    B, Hq, Hkv, D = 2, 32, 8, 128
+    scale = 1.0 / D ** 0.5
+    g = torch.Generator(device=dev)
+    res = {}
+    for N in (4096, 8192, 16384, 32768):
+        g.manual_seed(2000 + N)
+        q = torch.randn(B, N, Hq, D, device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn(B, N, Hkv, D, device=dev, generator=g)
+        k = (k * torch.where(torch.rand(B, N, Hkv, 1, device=dev, generator=g) < 0.01, 8.0, 1.0)).to(torch.bfloat16)
+        v = torch.randn(B, N, Hkv, D, device=dev, generator=g).to(torch.bfloat16)
+        out = torch.empty_like(q)
+        for W in sorted({1024, 4096, N}):
+            ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill(q, k, v, W, scale, out=out), iters), world)
+            tf = wl.useful_flops(B, N, W, Hq, D) / (ms * 1e-3) / 1e12
+            res[f"N{N}_W{W}" + ("_dense" if W == N else "")] = {"tflops": tf, "ms": ms}
+        del q, k, v, out
+    res["dense_over_swa_time_N16384_W4096"] = res["N16384_W16384_dense"]["ms"] / res["N16384_W4096"]["ms"]
+    return res
 
 
 def measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, iters, world):
