@@ -48,7 +48,10 @@ struct PrefillParams {
     int W;            // window (keys i-W < j <= i)
     int npairs;       // ceil(G / 2)
     int nqb;          // ceil(Nq / 128)
-    int num_units;    // B * Hkv * npairs * nqb
+    int num_units;    // B * Hkv * npairs * nqb, plus one per pair unit split in two
+    // pair units with index >= split_from are split into two single-head units
+    // (fills the last wave of CTAs; == the pair-unit count when nothing is split)
+    int split_from;
     float scale_log2; // softmax scale * log2(e)
     int chunk_mode;   // 1: keys also come from the rolling-buffer cache
     const int32_t *start_pos;  // chunk mode: [B] first position of the chunk
@@ -103,6 +106,7 @@ struct PrefillCfg {
 // Which query rows and key tiles one work unit covers.
 struct UnitPlan {
     int b, g, pair, qb;
+    int h0;          // query head of the unit's first head slot
     int q0;          // first query row (relative to the q tensor)
     int s0;          // absolute position of query row 0 of the sequence (chunk start, or 0)
     int qs;          // s0 mod W (slot the next position would take)
@@ -122,6 +126,7 @@ struct UnitPlan {
 __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, const int *pre) {
     constexpr int BM = 128, BN = 128;
     UnitPlan P;
+    int which = -1;
     if (p.cu_seqlens) {
         const int per = p.Hkv * p.npairs;
         const int qbi = pre[p.B] - 1 - u / per;        // later blocks first
@@ -141,9 +146,14 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         P.tb = 0;
         P.orow0 = (size_t)c0;
     } else {
+        int pu = u;                          // pair unit; which: head of a split unit
+        if (u >= p.split_from) {
+            pu = p.split_from + (u - p.split_from) / 2;
+            which = (u - p.split_from) & 1;
+        }
         const int per = p.B * p.Hkv * p.npairs;
-        P.qb = p.nqb - 1 - u / per;          // latest (heaviest) query blocks first
-        int r = u % per;
+        P.qb = p.nqb - 1 - pu / per;         // latest (heaviest) query blocks first
+        int r = pu % per;
         P.pair = r % p.npairs;
         r /= p.npairs;
         P.g = r % p.Hkv;
@@ -154,7 +164,8 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         P.orow0 = (size_t)P.b * p.Nq;
     }
     P.q0 = P.qb * BM;
-    P.act1 = (2 * P.pair + 1) < p.G;
+    P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
+    P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
     P.nc1 = P.nc2 = 0;
     P.c1 = P.c2 = 0;
     if (!p.chunk_mode) {
@@ -369,7 +380,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
                 mbar_arrive_expect_tx(bar_q_full, nact * TB);
                 for (int t = 0; t < nact; ++t) {
-                    const int h = P.g * p.G + 2 * P.pair + t;
+                    const int h = P.h0 + t;
                     for (int r = 0; r < NREG; ++r)
                         tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, P.row0 + P.q0, P.tb);
                 }
@@ -672,7 +683,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             ++oc;
             tc_fence_after();
-            const int h = P.g * p.G + 2 * P.pair + t;
+            const int h = P.h0 + t;
             const bool valid_row = i_rel < P.nq;
             const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
             __nv_bfloat16 *orow = p.out + ((P.orow0 + i_rel) * p.Hq + h) * D;

@@ -124,6 +124,20 @@ bool bad_scale(float s) { return !(std::isfinite(s) && s > 0.f); }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Chunk attention units (all about the same cost) fill whole waves of CTAs
+// except the last; when that wave is at most half full, its pair units are
+// split into two single-head units each, which fit in it and take about three
+// quarters of a pair unit's time.  Returns the first split pair unit and
+// raises units by the number split.
+int split_units(int &units, int G, int sms) {
+    if (G % 2 != 0 || units <= sms || units > 0x7fffffff - sms) return units;
+    const int rem = units % sms;
+    if (rem == 0 || 2 * rem > sms) return units;
+    const int from = units - rem;
+    units += rem;
+    return from;
+}
+
 template <int D>
 swa_status_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                             const CUtensorMap &mkc, const CUtensorMap &mvc,
@@ -296,6 +310,7 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.npairs = (G + 1) / 2;
     p.nqb = (int)nqb;
     p.num_units = (int)units;
+    p.split_from = cu_seqlens ? 0x7fffffff : (int)units;   // the lightest blocks come last: no split
     p.scale_log2 = scale * kLog2e;
     p.chunk_mode = 0;
     p.start_pos = nullptr;
@@ -352,6 +367,7 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     p.npairs = (G + 1) / 2;
     p.nqb = (int)nqb;
     p.num_units = (int)units;
+    p.split_from = cu_seqlens ? 0x7fffffff : split_units(p.num_units, G, dev->sms);
     p.scale_log2 = scale * kLog2e;
     p.chunk_mode = 1;
     p.start_pos = start_pos;
