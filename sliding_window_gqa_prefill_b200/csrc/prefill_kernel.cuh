@@ -214,6 +214,14 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
     return P;
 }
 
+// Unit taken by CTA c of C in round k: rounds alternate direction, so the
+// CTAs that drew the heavier units of one round draw the lighter ones of the
+// next (units are ordered heaviest first), which evens out the per-CTA work;
+// >= the unit count once the CTA has no more work.
+__device__ __forceinline__ int unit_of(int k, int c, int C) {
+    return k * C + ((k & 1) ? (C - 1 - c) : c);
+}
+
 // Key tile j of a unit: source (1 = cache), first row (slot or key index),
 // and whether any element of the 128x128 tile may be masked.
 struct TileRef {
@@ -374,7 +382,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             uint32_t k_cnt[KST] = {}, v_cnt[VST] = {};
             uint32_t q_cnt = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++uc) {
+            for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++uc) {
                 const UnitPlan P = plan_unit(p, u, pre);
                 const int nact = 1 + P.act1;
                 if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
@@ -431,7 +439,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             uint32_t pc[2] = {0, 0};
             uint32_t qr1 = 0;                      // units with a second query head
             bool ok = true;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++uc) {
+            for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++uc) {
                 const UnitPlan P = plan_unit(p, u, pre);
                 const int n = P.n;
                 if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
@@ -552,7 +560,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float sl2 = p.scale_log2;
         uint32_t sc = 0, oc = 0, qc = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++qc) {
+        for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++qc) {
             const UnitPlan P = plan_unit(p, u, pre);
             if (t == 1 && !P.act1) continue;
             const int i_rel = P.q0 + row;                  // query row in the q tensor
