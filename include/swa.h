@@ -211,6 +211,22 @@ swa_status_t swa_prefill_sinks(const void *q, const void *k, const void *v, void
                                int Hq, int Hkv, int D, int W, int S, float scale,
                                swa_stream_t stream);
 
+/* swa_prefill_chunk_sinks -- swa_prefill_chunk with S sink positions: each
+ * query at position i also attends to the sink positions j < S with
+ * j <= i - W (those that have left its window), read from the sink buffers
+ * k_sink / v_sink [B, S, Hkv, D], whose slot j must hold position j (written
+ * by an earlier chunk of this call family or by swa_cache_append_sinks).
+ * After the attention the chunk goes into the rolling buffer and its
+ * positions below S into the sink buffers.  A prompt pre-filled this way
+ * continues with swa_cache_append_sinks + swa_decode_sinks; the result equals
+ * swa_prefill_sinks over the whole prompt.  Fixed-length batches only; errors
+ * as swa_prefill_chunk, plus S < 0 or null / unaligned sink buffers with
+ * S > 0 -> SWA_ERR_INVALID_ARG. */
+swa_status_t swa_prefill_chunk_sinks(const void *q, const void *k, const void *v, void *k_cache,
+                                     void *v_cache, void *k_sink, void *v_sink, const int32_t *start_pos,
+                                     void *out, int B, int C, int Hq, int Hkv, int D, int W, int S,
+                                     float scale, swa_stream_t stream);
+
 /* swa_cache_append_sinks -- swa_cache_append that also stores new tokens
  * with position p < S at sink slot p. */
 swa_status_t swa_cache_append_sinks(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

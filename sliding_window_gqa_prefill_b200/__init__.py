@@ -95,7 +95,9 @@ def lib() -> ctypes.CDLL:
             L.swa_prefill_sinks.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, st]
             L.swa_cache_append_sinks.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, st]
             L.swa_decode_sinks.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, st]
-            for fn in (L.swa_prefill_sinks, L.swa_cache_append_sinks, L.swa_decode_sinks):
+            L.swa_prefill_chunk_sinks.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, st]
+            for fn in (L.swa_prefill_sinks, L.swa_cache_append_sinks, L.swa_decode_sinks,
+                       L.swa_prefill_chunk_sinks):
                 fn.restype = ctypes.c_int
             L.swa_decode_workspace_size.argtypes = [i, i, i, i, i]
             L.swa_decode_workspace_size.restype = ctypes.c_size_t
@@ -313,6 +315,25 @@ def swa_prefill_sinks(q, k, v, W: int, S: int, scale: float, out=None, stream=No
     _check(lib().swa_prefill_sinks(_bf16(q, "q"), _bf16(k, "k", (B, N, Hkv, D)), _bf16(v, "v", (B, N, Hkv, D)),
                                    _bf16(out, "out", (B, N, Hq, D)), B, N, Hq, Hkv, D, int(W), int(S), float(scale),
                                    _stream_handle(stream)), "swa_prefill_sinks")
+    return out
+
+
+def swa_prefill_chunk_sinks(q, k, v, k_cache, v_cache, k_sink, v_sink, start_pos, W: int, scale: float,
+                            out=None, stream=None):
+    """Chunked prefill of one chunk with the sink positions that left each
+    query's window read from the sink buffers [B,S,Hkv,D]; updates the cache
+    and the sink buffers (swa_prefill_chunk_sinks)."""
+    import torch
+    B, C, Hq, D = q.shape
+    Hkv, S = k.shape[2], k_sink.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().swa_prefill_chunk_sinks(
+        _bf16(q, "q"), _bf16(k, "k", (B, C, Hkv, D)), _bf16(v, "v", (B, C, Hkv, D)),
+        _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _bf16(k_sink, "k_sink", (B, S, Hkv, D)), _bf16(v_sink, "v_sink", (B, S, Hkv, D)),
+        _i32(start_pos, "start_pos", B), _bf16(out, "out", (B, C, Hq, D)), B, C, Hq, Hkv, D, int(W), int(S),
+        float(scale), _stream_handle(stream)), "swa_prefill_chunk_sinks")
     return out
 
 

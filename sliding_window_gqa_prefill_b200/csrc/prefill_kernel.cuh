@@ -64,6 +64,10 @@ struct PrefillParams {
     // attention sinks (one-shot prefill): positions j < sinks stay visible to
     // every query besides its window
     int sinks;
+    // attention sinks (chunk mode): slots 0 .. sink_buf-1 of the sink buffer
+    // hold positions 0 .. sink_buf-1; those outside a query's window are
+    // visible to it (0: no sinks)
+    int sink_buf;
 };
 
 constexpr int kMaxVarlenSeqs = 256;     // sequences per variable-length launch
@@ -114,7 +118,8 @@ struct UnitPlan {
     int nc1, c1;     // cache run 1: tiles c1 .. c1+nc1-1
     int nc2, c2;     // cache run 2
     int nm, m0;      // main tiles m0 .. m0+nm-1
-    int sink_tile;   // main tiles 0 .. sink_tile-1 below the band, visited first for the sinks
+    int sink_tile;   // sink tiles visited first: main tiles below the band (one-shot) or
+                     // sink-buffer tiles (chunk mode)
     int n;           // total tiles
     int nq;          // query rows of this sequence (== rows of its main k/v)
     int row0;        // first packed row of this sequence in q/k/v (varlen), else 0
@@ -178,12 +183,13 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         // sink positions below the band live in the first ceil(S/128) tiles
         P.sink_tile = min((p.sinks + BN - 1) / BN, P.m0);
     } else {
-        P.sink_tile = 0;
         P.s0 = __ldg(p.start_pos + P.b);
         if (P.s0 < 0) {                       // invalid start: record it, attend as if 0
             record_status(kStatusInvalid);
             P.s0 = 0;
         }
+        // sink positions j <= i - W exist for some row i of the block
+        P.sink_tile = (p.sink_buf > 0 && P.s0 + P.q0 + BM - 1 >= p.W) ? (p.sink_buf + BN - 1) / BN : 0;
         P.qs = P.s0 % p.W;
         // oldest age any row of the block still needs: age < W - q0, age <= s0
         const int A = min(p.W - P.q0 - 1, P.s0);
@@ -225,7 +231,7 @@ __device__ __forceinline__ int unit_of(int k, int c, int C) {
 // Key tile j of a unit: source (1 = cache), first row (slot or key index),
 // and whether any element of the 128x128 tile may be masked.
 struct TileRef {
-    int cache;
+    int cache;       // 0: main k/v, 1: rolling-buffer cache, 2: sink buffer (chunk mode)
     int row0;
     int masked;
 };
@@ -234,7 +240,7 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPl
     constexpr int BM = 128, BN = 128;
     TileRef t;
     if (j < P.sink_tile) {                  // only the sink positions of this tile count
-        t.cache = 0;
+        t.cache = p.chunk_mode ? 2 : 0;
         t.row0 = j * BN;
         t.masked = 1;
         return t;
@@ -283,6 +289,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_kc,
                    const __grid_constant__ CUtensorMap tm_vc,
+                   const __grid_constant__ CUtensorMap tm_ks,
+                   const __grid_constant__ CUtensorMap tm_vs,
                    const PrefillParams p) {
     using Cfg = PrefillCfg<D>;
     constexpr int BN = Cfg::BN, KST = Cfg::KST, VST = Cfg::VST;
@@ -364,6 +372,10 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             prefetch_tensormap(&tm_kc);
             prefetch_tensormap(&tm_vc);
         }
+        if (p.sink_buf > 0) {
+            prefetch_tensormap(&tm_ks);
+            prefetch_tensormap(&tm_vs);
+        }
     }
     if (warp == 2) {
         tmem_alloc(smem_addr(tmem_slot), Cfg::TMEM_COLS);
@@ -395,8 +407,8 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 ++q_cnt;
                 for (int j = 0; j < P.n; ++j) {
                     const TileRef T = tile_ref(p, P, j);
-                    const CUtensorMap *mk = T.cache ? &tm_kc : &tm_k;
-                    const CUtensorMap *mv = T.cache ? &tm_vc : &tm_v;
+                    const CUtensorMap *mk = T.cache == 2 ? &tm_ks : T.cache ? &tm_kc : &tm_k;
+                    const CUtensorMap *mv = T.cache == 2 ? &tm_vs : T.cache ? &tm_vc : &tm_v;
                     const uint32_t ks = kc % KST, kph = (kc / KST) & 1;
                     if (!mbar_wait_bounded(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, limit)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar_k_full + 8 * ks, TB);
@@ -600,7 +612,15 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 if (T.masked) {
-                    if (T.cache) {
+                    if (T.cache == 2) {
+                        // sink slot j holds position j: visible iff outside the window
+                        const int lim = P.s0 + i_rel - p.W;
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) {
+                            const int slot = T.row0 + c;
+                            if (slot >= p.sink_buf || slot > lim) s[c] = -INFINITY;
+                        }
+                    } else if (T.cache) {
                         // slot k0+c holds position s0 - age; valid iff age < W - t_rel, age <= s0
                         const int lim = min(p.W - i_rel - 1, P.s0);
 #pragma unroll

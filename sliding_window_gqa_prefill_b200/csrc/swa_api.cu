@@ -139,12 +139,13 @@ int split_units(int &units, int G, int sms) {
 }
 
 template <int D>
+// mks / mvs: sink-buffer maps (chunk mode with sinks), else any valid map.
 swa_status_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                            const CUtensorMap &mkc, const CUtensorMap &mvc,
-                            const swa::PrefillParams &p, int sms, cudaStream_t s) {
+                            const CUtensorMap &mkc, const CUtensorMap &mvc, const CUtensorMap &mks,
+                            const CUtensorMap &mvs, const swa::PrefillParams &p, int sms, cudaStream_t s) {
     const int grid = p.num_units < sms ? p.num_units : sms;
     swa::swa_prefill_kernel<D><<<grid, swa::PrefillCfg<D>::THREADS, swa::PrefillCfg<D>::SMEM_ALLOC, s>>>(
-        mq, mk, mv, mkc, mvc, p);
+        mq, mk, mv, mkc, mvc, mks, mvs, p);
     SWA_CUDA_TRY(cudaGetLastError());
     return SWA_OK;
 }
@@ -319,19 +320,23 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     if (rope) p.rope_freq = *rope;
     p.cu_seqlens = cu_seqlens;
     p.sinks = sinks;
-    return D == 128 ? launch_prefill<128>(mq, mk, mv, mk, mv, p, dev->sms, s)
-                    : launch_prefill<64>(mq, mk, mv, mk, mv, p, dev->sms, s);
+    return D == 128 ? launch_prefill<128>(mq, mk, mv, mk, mv, mk, mv, p, dev->sms, s)
+                    : launch_prefill<64>(mq, mk, mv, mk, mv, mk, mv, p, dev->sms, s);
 }
 
 // cu_seqlens non-null: variable-length batch; q/k/v/out packed [C = total rows,
 // H, D], sequence b is rows cu[b]..cu[b+1]-1 (any length; one longer than W
 // leaves its last W positions in the buffer).
+// k_sink / v_sink, S > 0: S-slot sink buffers [B, S, Hkv, D] (fixed-length only).
 swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, void *k_cache,
                                 void *v_cache, const int32_t *start_pos, void *out, int B, int C,
                                 int Hq, int Hkv, int D, int W, float scale,
                                 const swa::RopeTable *rope, const int32_t *cu_seqlens,
-                                cudaStream_t s) {
+                                cudaStream_t s, void *k_sink = nullptr, void *v_sink = nullptr,
+                                int S = 0) {
     if (!q || !k || !v || !k_cache || !v_cache || !start_pos || !out) return SWA_ERR_INVALID_ARG;
+    if (S < 0 || (S > 0 && (!k_sink || !v_sink || !aligned16(k_sink) || !aligned16(v_sink) || cu_seqlens)))
+        return SWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
         !aligned16(v_cache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
         return SWA_ERR_INVALID_ARG;
@@ -375,12 +380,19 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     p.rope = rope ? 1 : 0;
     if (rope) p.rope_freq = *rope;
     p.cu_seqlens = cu_seqlens;
-    swa_status_t e = D == 128 ? launch_prefill<128>(mq, mk, mv, mkc, mvc, p, dev->sms, s)
-                              : launch_prefill<64>(mq, mk, mv, mkc, mvc, p, dev->sms, s);
+    CUtensorMap mks = mkc, mvs = mvc;
+    if (S > 0) {
+        if (swa_status_t e = make_operand_map(&mks, k_sink, D, Hkv, S, B)) return e;
+        if (swa_status_t e = make_operand_map(&mvs, v_sink, D, Hkv, S, B)) return e;
+    }
+    p.sink_buf = S;
+    swa_status_t e = D == 128 ? launch_prefill<128>(mq, mk, mv, mkc, mvc, mks, mvs, p, dev->sms, s)
+                              : launch_prefill<64>(mq, mk, mv, mkc, mvc, mks, mvs, p, dev->sms, s);
     if (e) return e;
     // attend first, then write the chunk (its keys already rotated) into the buffer
-    if (!cu_seqlens)
-        return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, nullptr, s);
+    if (!cu_seqlens)     // positions below S also go to the sink buffer
+        return launch_append(k, v, k_cache, v_cache, start_pos, B, C, Hkv, D, W, dev->sms, nullptr, s,
+                             k_sink, v_sink, S);
     const int row_vec = Hkv * D * 2 / 16;
     long long blocks = ((long long)C * row_vec + 255) / 256;
     if (blocks > (long long)dev->sms * 8) blocks = (long long)dev->sms * 8;
@@ -576,6 +588,14 @@ swa_status_t swa_prefill_sinks(const void *q, const void *k, const void *v, void
     if (S < 0) return SWA_ERR_INVALID_ARG;
     return prefill_impl(q, k, v, out, B, N, Hq, Hkv, D, W, SWA_WINDOW_EXCL_LEFT, scale, nullptr, nullptr,
                         reinterpret_cast<cudaStream_t>(stream), S);
+}
+
+swa_status_t swa_prefill_chunk_sinks(const void *q, const void *k, const void *v, void *k_cache,
+                                     void *v_cache, void *k_sink, void *v_sink, const int32_t *start_pos,
+                                     void *out, int B, int C, int Hq, int Hkv, int D, int W, int S,
+                                     float scale, swa_stream_t stream) {
+    return prefill_chunk_impl(q, k, v, k_cache, v_cache, start_pos, out, B, C, Hq, Hkv, D, W, scale,
+                              nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream), k_sink, v_sink, S);
 }
 
 swa_status_t swa_cache_append_sinks(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -60,6 +60,11 @@ def test_null_and_bad_sizes_rejected_without_device(lib):
     # append: T > W, null pos
     assert lib.swa_cache_append(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, 1, 65, 2, 128, 64, None) == S
     assert lib.swa_cache_append(ok_ptr, ok_ptr, ok_ptr, ok_ptr, null, 1, 1, 2, 128, 64, None) == S
+    # chunked prefill with sinks: negative S, null sink buffer with S > 0
+    assert lib.swa_prefill_chunk_sinks(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr,
+                                       1, 128, 8, 2, 128, 256, -1, 0.1, None) == S
+    assert lib.swa_prefill_chunk_sinks(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, null, ok_ptr, ok_ptr, ok_ptr,
+                                       1, 128, 8, 2, 128, 256, 4, 0.1, None) == S
     # decode: workspace too small
     assert lib.swa_decode(ok_ptr, ok_ptr, ok_ptr, ok_ptr, ok_ptr, 2, 8, 2, 128, 4096, 0.1,
                           ok_ptr, 16, None) == S

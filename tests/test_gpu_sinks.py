@@ -79,3 +79,45 @@ def test_streaming_decode_with_sinks(oracle_mod, W, S, D):
             close(out.cpu(), ref, f"decode sinks step {p}")
     torch.cuda.synchronize()
     assert np.array_equal(f64(ks.cpu()), ksr) and np.array_equal(f64(ks.cpu()), f64(k[:S].permute(1, 0, 2, 3)))
+
+
+@pytest.mark.parametrize("B,N,C,Hq,Hkv,D,W,S", [
+    (1, 900, 256, 8, 2, 128, 256, 4),     # C = W
+    (2, 700, 100, 4, 4, 64, 128, 8),      # C < W, MHA, D=64
+    (1, 1000, 300, 6, 2, 128, 384, 130),  # two sink tiles, odd group
+])
+def test_chunked_prefill_with_sinks(oracle_mod, B, N, C, Hq, Hkv, D, W, S):
+    """Chunks through the rolling buffer with the sink buffer: the outputs equal
+    one-shot prefill with sinks over the whole prompt; afterwards the sink
+    buffer holds positions 0..S-1 and the cache the last W positions, bit for
+    bit; decode with sinks then continues the sequence."""
+    q = wl.random_bf16((B, N + 2, Hq, D), 111)
+    k = wl.random_bf16((B, N + 2, Hkv, D), 112)
+    v = wl.random_bf16((B, N + 2, Hkv, D), 113)
+    scale = 1 / math.sqrt(D)
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ks = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vs = torch.zeros_like(ks)
+    outs = []
+    for s0 in range(0, N, C):
+        e = min(N, s0 + C)
+        st = torch.full((B,), s0, dtype=torch.int32, device="cuda")
+        outs.append(swa.swa_prefill_chunk_sinks(q[:, s0:e].cuda().contiguous(), k[:, s0:e].cuda().contiguous(),
+                                                v[:, s0:e].cuda().contiguous(), kc, vc, ks, vs, st, W, scale))
+    torch.cuda.synchronize()
+    ref = oracle_mod.swa_prefill_sinks(f64(q), f64(k), f64(v), W, S, scale)
+    close(torch.cat([o.cpu() for o in outs], dim=1), ref[:, :N], f"chunked sinks W{W} S{S}")
+    assert torch.equal(ks.cpu(), k[:, :S]) and torch.equal(vs.cpu(), v[:, :S])
+    for slot in range(W):
+        p = slot + ((N - 1 - slot) // W) * W
+        assert torch.equal(kc[:, slot].cpu(), k[:, p]) and torch.equal(vc[:, slot].cpu(), v[:, p]), slot
+    if Hq // Hkv not in (1, 2, 4, 8):      # decode takes these group sizes (SWA_ERR_UNSUPPORTED otherwise)
+        return
+    for p in (N, N + 1):
+        pos = torch.full((B,), p, dtype=torch.int32, device="cuda")
+        swa.swa_cache_append_sinks(k[:, p:p + 1].cuda().contiguous(), v[:, p:p + 1].cuda().contiguous(), kc, vc,
+                                   ks, vs, pos)
+        out = swa.swa_decode_sinks(q[:, p].cuda().contiguous(), kc, vc, ks, vs, pos, scale)
+        torch.cuda.synchronize()
+        close(out.cpu(), ref[:, p], f"decode with sinks after chunks at {p}")
