@@ -562,6 +562,23 @@ def measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, iters, world):
     sflops = flops + 4 * hp.B * hp.Hq * hp.D * sink_pairs
     ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill_sinks(q, k, v, hp.W, S, hp.scale, out=out), iters), world)
     res["prefill_sinks4"] = {"tflops": sflops / ms / 1e9, "ms": ms}
+    # the same prompt (sequence 0) pre-filled in chunks of W with 4 sinks
+    C = hp.W
+    cqs = [(q[:1, s0:s0 + C].contiguous(), k[:1, s0:s0 + C].contiguous(), v[:1, s0:s0 + C].contiguous())
+           for s0 in range(0, hp.N, C)]
+    cst = [torch.full((1,), s0, dtype=torch.int32, device=dev) for s0 in range(0, hp.N, C)]
+    ckc = torch.zeros(1, hp.W, hp.Hkv, hp.D, dtype=torch.bfloat16, device=dev)
+    cvc = torch.zeros_like(ckc)
+    cks = torch.zeros(1, S, hp.Hkv, hp.D, dtype=torch.bfloat16, device=dev)
+    cvs = torch.zeros_like(cks)
+    couts = [torch.empty_like(a) for a, _, _ in cqs]
+
+    def chunks_sinks():
+        for (a, b_, c), st, o in zip(cqs, cst, couts):
+            swa.swa_prefill_chunk_sinks(a, b_, c, ckc, cvc, cks, cvs, st, hp.W, hp.scale, out=o)
+
+    ms = max_over_ranks(_time_ms(chunks_sinks, iters), world)
+    res["chunked_sinks4_B1"] = {"tflops": sflops / hp.B / ms / 1e9, "ms": ms, "chunks": len(cqs)}
     # decode with fused RoPE and with sinks: one step at B=64 (append + decode)
     kc, vc = dd["k_cache"].to(dev), dd["v_cache"].to(dev)
     ks = torch.zeros(dw.B, S, dw.Hkv, dw.D, dtype=torch.bfloat16, device=dev)
