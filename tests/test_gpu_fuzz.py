@@ -43,7 +43,7 @@ def _heads(rng):
     return Hkv * G, Hkv, int(rng.choice([64, 128]))
 
 
-@pytest.mark.parametrize("case", range(10))
+@pytest.mark.parametrize("case", range(16))
 def test_fuzz_prefill(oracle_mod, case):
     rng = np.random.default_rng(9000 + case)
     B = int(rng.integers(1, 4))
@@ -61,7 +61,7 @@ def test_fuzz_prefill(oracle_mod, case):
     close(out, ref, f"prefill B{B} N{N} W{W} H{Hq}/{Hkv} D{D}")
 
 
-@pytest.mark.parametrize("case", range(8))
+@pytest.mark.parametrize("case", range(12))
 def test_fuzz_chunked(oracle_mod, case):
     rng = np.random.default_rng(9500 + case)
     B = int(rng.integers(1, 3))
@@ -90,7 +90,7 @@ def test_fuzz_chunked(oracle_mod, case):
         assert torch.equal(kc[:, slot].cpu(), k[:, p]) and torch.equal(vc[:, slot].cpu(), v[:, p]), slot
 
 
-@pytest.mark.parametrize("case", range(8))
+@pytest.mark.parametrize("case", range(12))
 def test_fuzz_decode(oracle_mod, case):
     rng = np.random.default_rng(9800 + case)
     B = int(rng.integers(1, 6))
@@ -119,3 +119,96 @@ def test_fuzz_decode(oracle_mod, case):
         ref = oracle_mod.swa_decode(f64(q), kr, vr, sp, pos.numpy(), W, scale)
         close(out.cpu(), ref, f"decode B{B} W{W} H{Hq}/{Hkv} D{D} step {s}")
     assert np.array_equal(f64(kg.cpu()), kr) and np.array_equal(f64(vg.cpu()), vr)
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_fuzz_varlen(oracle_mod, case):
+    """Packed batch of random lengths (zeros included): each sequence equals its own one-shot prefill."""
+    rng = np.random.default_rng(10100 + case)
+    lens = [int(x) for x in rng.integers(0, 600, size=int(rng.integers(1, 7)))]
+    lens[int(rng.integers(0, len(lens)))] = max(1, lens[0])
+    W = int(rng.integers(1, 650))
+    Hq, Hkv, D = _heads(rng)
+    total = sum(lens)
+    cu = np.array([0] + list(np.cumsum(lens)), np.int32)
+    seed = 10200 + 10 * case
+    q = wl.random_bf16((total, Hq, D), seed)
+    k = wl.random_bf16((total, Hkv, D), seed + 1)
+    v = wl.random_bf16((total, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    out = swa.swa_prefill_varlen(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cu).cuda(), W, scale)
+    torch.cuda.synchronize()
+    out = out.cpu()
+    for b, n in enumerate(lens):
+        s, e = int(cu[b]), int(cu[b + 1])
+        if n == 0:
+            continue
+        ref = oracle_mod.swa_prefill(f64(q[s:e])[None], f64(k[s:e])[None], f64(v[s:e])[None], W, scale)
+        close(out[s:e], ref[0], f"varlen seq {b} n{n} W{W} H{Hq}/{Hkv} D{D}")
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_fuzz_mixed_chunk_varlen(oracle_mod, case):
+    """One packed call continuing several sequences from random histories (decode-length pieces included)."""
+    rng = np.random.default_rng(10500 + case)
+    B = int(rng.integers(1, 6))
+    W = int(rng.integers(8, 700))
+    Hq, Hkv, D = _heads(rng)
+    hist = [int(x) for x in rng.integers(0, 3 * W, size=B)]
+    now = [int(x) for x in rng.integers(0, W + 1, size=B)]
+    now[0] = max(now[0], 1)
+    seed = 10600 + 10 * case
+    kref = np.zeros((B, W, Hkv, D))
+    vref = np.zeros_like(kref)
+    sp = np.full((B, W), -1, np.int32)
+    for b in range(B):
+        if hist[b]:
+            kh = f64(wl.random_bf16((1, hist[b], Hkv, D), seed + 100 + b))
+            vh = f64(wl.random_bf16((1, hist[b], Hkv, D), seed + 200 + b))
+            kb, vb, spb = kref[b:b + 1].copy(), vref[b:b + 1].copy(), sp[b:b + 1].copy()
+            oracle_mod.cache_append(kb, vb, spb, kh[:, -W:], vh[:, -W:], [max(0, hist[b] - W)])
+            kref[b], vref[b], sp[b] = kb[0], vb[0], spb[0]
+    total = sum(now)
+    cu = np.array([0] + list(np.cumsum(now)), np.int32)
+    q = wl.random_bf16((total, Hq, D), seed)
+    k = wl.random_bf16((total, Hkv, D), seed + 1)
+    v = wl.random_bf16((total, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    kg = torch.from_numpy(kref).to(torch.bfloat16).cuda()
+    vg = torch.from_numpy(vref).to(torch.bfloat16).cuda()
+    out = swa.swa_prefill_chunk_varlen(q.cuda(), k.cuda(), v.cuda(), kg, vg,
+                                       torch.tensor(hist, dtype=torch.int32).cuda(),
+                                       torch.from_numpy(cu).cuda(), W, scale)
+    torch.cuda.synchronize()
+    out = out.cpu()
+    for b in range(B):
+        s, e = int(cu[b]), int(cu[b + 1])
+        if e == s:
+            continue
+        ref = oracle_mod.swa_chunk(f64(q[s:e])[None], f64(k[s:e])[None], f64(v[s:e])[None],
+                                   kref[b:b + 1], vref[b:b + 1], sp[b:b + 1], [hist[b]], W, scale)
+        close(out[s:e], ref[0], f"mixed seq {b} hist{hist[b]} n{e - s} W{W} H{Hq}/{Hkv} D{D}")
+        kb, vb = kref[b:b + 1].copy(), vref[b:b + 1].copy()
+        oracle_mod.cache_append(kb, vb, None, f64(k[s:e])[None], f64(v[s:e])[None], [hist[b]])
+        kref[b], vref[b] = kb[0], vb[0]
+    assert np.array_equal(f64(kg.cpu()), kref) and np.array_equal(f64(vg.cpu()), vref)
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_fuzz_sinks(oracle_mod, case):
+    """One-shot prefill with S sink positions; S below, inside and beyond the window and the sequence."""
+    rng = np.random.default_rng(10900 + case)
+    B = int(rng.integers(1, 3))
+    N = int(rng.integers(1, 800))
+    W = int(rng.integers(1, N + 40))
+    S = int(rng.integers(0, N + 20))
+    Hq, Hkv, D = _heads(rng)
+    seed = 11000 + 10 * case
+    q = wl.random_bf16((B, N, Hq, D), seed)
+    k = wl.random_bf16((B, N, Hkv, D), seed + 1)
+    v = wl.random_bf16((B, N, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    out = swa.swa_prefill_sinks(q.cuda(), k.cuda(), v.cuda(), W, S, scale)
+    torch.cuda.synchronize()
+    ref = oracle_mod.swa_prefill_sinks(f64(q), f64(k), f64(v), W, S, scale)
+    close(out, ref, f"sinks B{B} N{N} W{W} S{S} H{Hq}/{Hkv} D{D}")
