@@ -56,6 +56,7 @@ struct PrefillParams {
     int chunk_mode;   // 1: keys also come from the rolling-buffer cache
     const int32_t *start_pos;  // chunk mode: [B] first position of the chunk
     __nv_bfloat16 *out;        // [B, Nq, Hq, D]
+    int out_v8;                // 1: out is 32-byte aligned (rows of 128 or 256 bytes): 32-byte stores
     int rope;                  // 1: rotate each Q tile in shared memory after its load
     RopeTable rope_freq;       // theta^(-2i/D), i < D/2
     // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
@@ -725,7 +726,13 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int e = 0; e < 16; ++e)
                     pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
                                         __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (valid_row) {
+                // each thread writes its own row (rows are Hq*D*2 bytes apart), so
+                // every store instruction touches 32 lines: wider stores mean fewer
+                // of them, which shortens the epilogue between units
+                if (valid_row && p.out_v8) {
+                    st_global_v8(orow + c * 32, pk);
+                    st_global_v8(orow + c * 32 + 16, pk + 8);
+                } else if (valid_row) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4)

@@ -316,6 +316,7 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.chunk_mode = 0;
     p.start_pos = nullptr;
     p.out = static_cast<__nv_bfloat16 *>(out);
+    p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     p.rope = rope ? 1 : 0;
     if (rope) p.rope_freq = *rope;
     p.cu_seqlens = cu_seqlens;
@@ -377,6 +378,7 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     p.chunk_mode = 1;
     p.start_pos = start_pos;
     p.out = static_cast<__nv_bfloat16 *>(out);
+    p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     p.rope = rope ? 1 : 0;
     if (rope) p.rope_freq = *rope;
     p.cu_seqlens = cu_seqlens;

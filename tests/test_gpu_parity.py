@@ -150,6 +150,36 @@ def test_dense_control_equals_wide_window():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_output_only_16_byte_aligned(D):
+    """An output 16 but not 32 bytes aligned takes the 16-byte store path of the
+    epilogue: same bits as a 32-byte aligned output, one-shot and chunked."""
+    B, N, Hq, Hkv, W = 2, 300, 8, 2, 200
+    q = wl.random_bf16((B, N, Hq, D), 41).cuda()
+    k = wl.random_bf16((B, N, Hkv, D), 42).cuda()
+    v = wl.random_bf16((B, N, Hkv, D), 43).cuda()
+    n = B * N * Hq * D
+    flat = torch.zeros(n + 16, dtype=torch.bfloat16, device="cuda")
+    assert flat.data_ptr() % 32 == 0
+    odd = flat[8:8 + n].view(B, N, Hq, D)            # 16 bytes past a 32-byte boundary
+    ref = swa.swa_prefill(q, k, v, W, 0.1)
+    swa.swa_prefill(q, k, v, W, 0.1, out=odd)
+    torch.cuda.synchronize()
+    assert torch.equal(odd, ref)
+    assert not flat[:8].any() and not flat[8 + n:].any()
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    st = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ref_c = swa.swa_prefill_chunk(q[:, :150].contiguous(), k[:, :150].contiguous(), v[:, :150].contiguous(),
+                                  kc.clone(), vc.clone(), st, W, 0.1)
+    m = B * 150 * Hq * D
+    odd_c = flat[8:8 + m].view(B, 150, Hq, D)
+    swa.swa_prefill_chunk(q[:, :150].contiguous(), k[:, :150].contiguous(), v[:, :150].contiguous(),
+                          kc, vc, st, W, 0.1, out=odd_c)
+    torch.cuda.synchronize()
+    assert torch.equal(odd_c, ref_c)
+
+
 # ------------------------------------------------------------------ rolling buffer append
 
 @pytest.mark.parametrize("B,T,Hkv,D,W", [(3, 1, 8, 128, 64), (2, 37, 2, 64, 50), (1, 64, 4, 128, 64),
