@@ -24,7 +24,7 @@
  *       behind i), section 3 (rolling buffer, i mod W), section 4 (pre-fill
  *       and chunking: attention over the current chunk and the active cache).
  *
- * Readings taken where the pages are loose (all listed in the design doc):
+ * Readings taken where the sources above are loose or disagree:
  *  - window: query i sees keys j with i-W < j <= i (W keys, itself included).
  *    The other printed reading, i-W <= j <= i (W+1 keys), is window_mode 1.
  *  - GQA grouping is contiguous: query head h uses KV head h / (Hq/Hkv).
