@@ -212,3 +212,100 @@ def test_fuzz_sinks(oracle_mod, case):
     torch.cuda.synchronize()
     ref = oracle_mod.swa_prefill_sinks(f64(q), f64(k), f64(v), W, S, scale)
     close(out, ref, f"sinks B{B} N{N} W{W} S{S} H{Hq}/{Hkv} D{D}")
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_fuzz_rope_sequence(oracle_mod, case):
+    """RoPE: one-shot prefill with q rotated in the kernel, the same prompt in
+    chunks, then two decode steps with the key rotated on its way into the
+    cache; every output equals SWA on exactly rotated q and k."""
+    rng = np.random.default_rng(11500 + case)
+    B = int(rng.integers(1, 3))
+    W = int(rng.integers(16, 500))
+    C = int(rng.integers(1, W + 1))
+    N = int(rng.integers(C, 3 * W))
+    Hkv = int(rng.choice([1, 2, 4]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    Hq, D = Hkv * G, int(rng.choice([64, 128]))
+    theta = float(rng.choice([10000.0, 1000000.0]))
+    seed = 11600 + 10 * case
+    q = wl.random_bf16((B, N + 2, Hq, D), seed)
+    k = wl.random_bf16((B, N + 2, Hkv, D), seed + 1)
+    v = wl.random_bf16((B, N + 2, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    zero = torch.zeros(B, dtype=torch.int32, device="cuda")
+    kr_dev = k[:, :N].cuda().contiguous()
+    swa.swa_rope(kr_dev, zero, theta)
+    one = swa.swa_prefill(q[:, :N].cuda().contiguous(), kr_dev, v[:, :N].cuda().contiguous(), W, scale,
+                          rope_theta=theta)
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    outs = []
+    for s0 in range(0, N, C):
+        e = min(N, s0 + C)
+        st = torch.full((B,), s0, dtype=torch.int32, device="cuda")
+        kch = k[:, s0:e].cuda().contiguous()
+        swa.swa_rope(kch, st, theta)
+        outs.append(swa.swa_prefill_chunk(q[:, s0:e].cuda().contiguous(), kch, v[:, s0:e].cuda().contiguous(),
+                                          kc, vc, st, W, scale, rope_theta=theta))
+    dec = []
+    for p in (N, N + 1):
+        pos = torch.full((B,), p, dtype=torch.int32, device="cuda")
+        swa.swa_cache_append(k[:, p:p + 1].cuda().contiguous(), v[:, p:p + 1].cuda().contiguous(), kc, vc, pos,
+                             rope_theta=theta)
+        dec.append(swa.swa_decode(q[:, p].cuda().contiguous(), kc, vc, pos, scale, rope_theta=theta))
+    torch.cuda.synchronize()
+    z = np.zeros(B, np.int32)
+    ref = oracle_mod.swa_prefill(oracle_mod.rope(f64(q), z, theta), oracle_mod.rope(f64(k), z, theta), f64(v),
+                                 W, scale)
+    tag = f"rope B{B} N{N} C{C} W{W} H{Hq}/{Hkv} D{D} theta{theta:g}"
+    close(one, ref[:, :N], "one-shot " + tag)
+    close(torch.cat([o.cpu() for o in outs], dim=1), ref[:, :N], "chunked " + tag)
+    for i, p in enumerate((N, N + 1)):
+        close(dec[i].cpu(), ref[:, p], f"decode at {p} " + tag)
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_fuzz_sinks_sequence(oracle_mod, case):
+    """Sinks: the prompt in chunks through the rolling buffer and the sink
+    buffer, then two decode steps with sinks; outputs equal one-shot prefill
+    with sinks over the whole sequence, buffers bit for bit."""
+    rng = np.random.default_rng(11800 + case)
+    B = int(rng.integers(1, 3))
+    W = int(rng.integers(8, 400))
+    C = int(rng.integers(1, W + 1))
+    N = int(rng.integers(C, 3 * W + 2))
+    S = int(rng.integers(1, min(N, 300) + 1))
+    Hkv = int(rng.choice([1, 2, 4]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    Hq, D = Hkv * G, int(rng.choice([64, 128]))
+    seed = 11900 + 10 * case
+    q = wl.random_bf16((B, N + 2, Hq, D), seed)
+    k = wl.random_bf16((B, N + 2, Hkv, D), seed + 1)
+    v = wl.random_bf16((B, N + 2, Hkv, D), seed + 2)
+    scale = 1.0 / math.sqrt(D)
+    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ks = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    vs = torch.zeros_like(ks)
+    outs = []
+    for s0 in range(0, N, C):
+        e = min(N, s0 + C)
+        st = torch.full((B,), s0, dtype=torch.int32, device="cuda")
+        outs.append(swa.swa_prefill_chunk_sinks(q[:, s0:e].cuda().contiguous(), k[:, s0:e].cuda().contiguous(),
+                                                v[:, s0:e].cuda().contiguous(), kc, vc, ks, vs, st, W, scale))
+    torch.cuda.synchronize()
+    ref = oracle_mod.swa_prefill_sinks(f64(q), f64(k), f64(v), W, S, scale)
+    tag = f"sinks B{B} N{N} C{C} W{W} S{S} H{Hq}/{Hkv} D{D}"
+    close(torch.cat([o.cpu() for o in outs], dim=1), ref[:, :N], "chunked " + tag)
+    assert torch.equal(ks.cpu(), k[:, :S]) and torch.equal(vs.cpu(), v[:, :S]), tag
+    for p in (N, N + 1):
+        pos = torch.full((B,), p, dtype=torch.int32, device="cuda")
+        swa.swa_cache_append_sinks(k[:, p:p + 1].cuda().contiguous(), v[:, p:p + 1].cuda().contiguous(), kc, vc,
+                                   ks, vs, pos)
+        out = swa.swa_decode_sinks(q[:, p].cuda().contiguous(), kc, vc, ks, vs, pos, scale)
+        torch.cuda.synchronize()
+        close(out.cpu(), ref[:, p], f"decode at {p} " + tag)
+    for slot in range(min(W, N + 2)):
+        p = slot + ((N + 1 - slot) // W) * W
+        assert torch.equal(kc[:, slot].cpu(), k[:, p]) and torch.equal(vc[:, slot].cpu(), v[:, p]), (tag, slot)
