@@ -17,9 +17,12 @@ import threading
 
 __all__ = [
     "SwaError", "build", "lib", "swa_prefill", "swa_prefill_chunk", "swa_cache_append",
-    "swa_decode", "swa_decode_workspace_size", "swa_get_device_status", "swa_set_wait_limit_ns",
-    "swa_selftest_wait_timeout", "swa_rope", "SWA_OK", "SWA_ERR_INVALID_ARG", "SWA_ERR_UNSUPPORTED",
-    "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_WINDOW_EXCL_LEFT", "SWA_WINDOW_INCL_LEFT",
+    "swa_decode", "swa_decode_workspace_size", "swa_decode_noalloc", "swa_prefill_varlen",
+    "swa_prefill_chunk_varlen", "swa_prefill_sinks", "swa_prefill_chunk_sinks", "swa_cache_append_sinks",
+    "swa_decode_sinks", "swa_rope", "swa_get_device_status", "swa_set_wait_limit_ns",
+    "swa_selftest_wait_timeout", "swa_selftest_exp2", "SWA_OK", "SWA_ERR_INVALID_ARG",
+    "SWA_ERR_UNSUPPORTED", "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_WINDOW_EXCL_LEFT",
+    "SWA_WINDOW_INCL_LEFT",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -243,6 +246,20 @@ def swa_decode(q, k_cache, v_cache, pos, scale: float, out=None, workspace=None,
         _check(lib().swa_decode(*head, *tail), "swa_decode")
     else:
         _check(lib().swa_decode_rope(*head, float(rope_theta), *tail), "swa_decode_rope")
+    return out
+
+
+def swa_decode_noalloc(q, k_cache, v_cache, pos, scale: float, out, stream=None):
+    """Decode like swa_decode with the split partials in the library's static
+    device scratch (SWA_DECODE_NOALLOC_SCRATCH_BYTES): nothing is allocated, so
+    out [B,Hq,D] must be given.  Calls that overlap on the GPU share that one
+    scratch array and race: serialise them."""
+    B, Hq, D = q.shape
+    W, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _check(lib().swa_decode_noalloc(
+        _bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)), _i32(pos, "pos", B),
+        _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale), _stream_handle(stream)),
+        "swa_decode_noalloc")
     return out
 
 

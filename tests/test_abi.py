@@ -78,3 +78,31 @@ def test_workspace_size_and_status_strings(lib):
     assert n == ((rows * 128 * 4 + 255) // 256) * 256 + rows * 8
     assert lib.swa_status_string(0) == b"SWA_OK"
     assert lib.swa_status_string(4) == b"SWA_ERR_TIMEOUT"
+
+
+def test_every_declared_operation_has_a_python_binding():
+    """Each symbol of include/swa.h is reachable from Python: a wrapper of the
+    same name, the rope_theta argument of the base wrapper for the *_rope
+    entry points, or the error path (status string, last CUDA error)."""
+    import inspect
+    src = inspect.getsource(swa)
+    for name in declared_symbols():
+        if hasattr(swa, name):
+            continue
+        if name.endswith("_rope") and hasattr(swa, name[:-5]):
+            assert "rope_theta" in inspect.signature(getattr(swa, name[:-5])).parameters, name
+            assert f"lib().{name}(" in src, name
+            continue
+        assert name in ("swa_status_string", "swa_last_cuda_error"), name
+        assert f".{name}(" in src, name
+    for name in swa.__all__:
+        assert hasattr(swa, name), name
+
+
+def test_noalloc_binding_checks_its_arguments_on_the_host():
+    import torch
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(2, 64, 2, 128, dtype=torch.bfloat16)
+    pos = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(TypeError):
+        swa.swa_decode_noalloc(q, kc, kc, pos, 0.1, out=torch.empty_like(q))

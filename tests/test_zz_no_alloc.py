@@ -70,3 +70,21 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert swa.swa_decode_workspace_size(B, Hq, Hkv, D, W) > (16 << 20)
     st = L.swa_decode_noalloc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, B, Hq, Hkv, D, W, 0.1, None)
     assert st == swa.SWA_ERR_UNSUPPORTED
+
+
+def test_noalloc_python_binding_matches_the_c_call():
+    """The Python binding passes its arguments through unchanged: same bits as
+    the raw C call on the same inputs."""
+    swa.build()
+    L = swa.lib()
+    B, Hq, Hkv, D, W = 8, 32, 8, 128, 4096
+    scale = 1.0 / math.sqrt(D)
+    q, kc, vc, pos = _inputs(B, Hq, Hkv, D, W, 303)
+    a = torch.empty_like(q)
+    b = swa.swa_decode_noalloc(q, kc, vc, pos, scale, torch.empty_like(q))
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = L.swa_decode_noalloc(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), pos.data_ptr(), a.data_ptr(),
+                              B, Hq, Hkv, D, W, scale, stream)
+    assert st == swa.SWA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
