@@ -14,7 +14,9 @@
  * Conventions shared by every call
  *  - Tensors are caller-owned DEVICE memory, bfloat16 (stored as uint16_t),
  *    contiguous row-major, with the shapes given per call.  Every tensor base
- *    address must be 16-byte aligned.  The library never allocates, frees or
+ *    address must be 16-byte aligned; a prefill output that is 32-byte
+ *    aligned is written with 32-byte stores (same values, fewer store
+ *    instructions).  The library never allocates, frees or
  *    retains them; it never synchronises a stream except in
  *    swa_get_device_status().
  *  - Positions are 0-based int32 values in DEVICE memory, so a sequence of
