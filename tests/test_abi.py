@@ -106,3 +106,26 @@ def test_noalloc_binding_checks_its_arguments_on_the_host():
     pos = torch.zeros(2, dtype=torch.int32)
     with pytest.raises(TypeError):
         swa.swa_decode_noalloc(q, kc, kc, pos, 0.1, out=torch.empty_like(q))
+
+
+def test_product_path_does_not_use_the_oracle():
+    """The package and its C sources never import, load or link the oracle;
+    bench.py reaches it only in the CPU-baseline sampler that its cpu_baseline
+    leg and its reference arm call."""
+    import ast
+    pkg = os.path.join(ROOT, "sliding_window_gqa_prefill_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in text and "libswa_oracle" not in text, f
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    users = set()
+    for fn in ast.walk(tree):
+        if isinstance(fn, ast.FunctionDef):
+            for node in ast.walk(fn):
+                if isinstance(node, ast.Import) and any(a.name == "oracle" for a in node.names):
+                    users.add(fn.name)
+    top_level = [n for n in tree.body if isinstance(n, (ast.Import, ast.ImportFrom))
+                 and any(a.name == "oracle" for a in n.names)]
+    assert not top_level and users == {"cpu_oracle_sample"}, users
