@@ -80,7 +80,10 @@ struct PrefillCfg {
     static constexpr int NREG = D / 64;            // 64-column (128-byte) swizzle regions
     static constexpr int REGION_BYTES = 128 * 128; // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = NREG * REGION_BYTES;
-    static constexpr int KST = 3;                  // K ring depth
+    // K ring depth: 2 measured 1-5% faster than 3; the 32 KB it frees leave
+    // more of the SM's unified L1 / shared storage to L1, through which the
+    // softmax warps' register spills go
+    static constexpr int KST = 2;
     static constexpr int VST = 2;                  // V ring depth
     static constexpr int OFF_Q = 0;                // two Q tiles
     static constexpr int OFF_K = 2 * TILE_BYTES;
