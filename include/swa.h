@@ -125,7 +125,10 @@ swa_status_t swa_cache_append(const void *k_new, const void *v_new,
  *   pos : int32 [B] device array, position of the new token, whose K/V must
  *         already be in the cache (swa_cache_append first).
  * Each sequence reads slots 0 .. min(pos[b]+1, W)-1; softmax is order-free,
- * so the wrap needs no reordering.
+ * so the wrap needs no reordering.  Group sizes Hq/Hkv of 1, 2, 4 and 8 are
+ * covered (Mistral-7B: 4); others return SWA_ERR_UNSUPPORTED, as do the
+ * _rope, _sinks and _noalloc forms.  (A decode step of any group size runs
+ * through swa_prefill_chunk_varlen as a length-1 sequence.)
  * workspace: device scratch of at least swa_decode_workspace_size() bytes,
  *   256-byte aligned, owned by the caller; its contents need no set-up and are
  *   overwritten.  Calls that share a workspace must not overlap on the GPU.
