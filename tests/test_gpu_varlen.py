@@ -55,8 +55,9 @@ def test_prefill_varlen_matches_per_sequence_oracle(oracle_mod, lens, Hq, Hkv, D
         close(out[s:e], ref[0], f"varlen seq {b} (n={n})")
 
 
-def test_mixed_chunks_and_decode_in_one_launch(oracle_mod):
-    Hq, Hkv, D, W = 8, 2, 128, 256
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (6, 2), (6, 1)])   # group sizes 4, 3 and 6
+def test_mixed_chunks_and_decode_in_one_launch(oracle_mod, Hq, Hkv):
+    D, W = 128, 256
     scale = 1 / math.sqrt(D)
     # per sequence: history length already in the buffer, tokens in this call
     hist = [1000, 7000, 0, 300, 50]
