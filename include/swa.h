@@ -21,6 +21,10 @@
  *    swa_get_device_status().
  *  - Positions are 0-based int32 values in DEVICE memory, so a sequence of
  *    calls can be captured in a CUDA graph and replayed with new positions.
+ *    Every position a call covers (start + length - 1) must fit in int32;
+ *    a negative position is recorded as SWA_ERR_INVALID_ARG in the device
+ *    status word (appends, RoPE and decode then skip that sequence; chunked
+ *    prefill attends as if the chunk started at position 0).
  *  - Window: query position i attends to key positions j with i-W < j <= i
  *    (W keys, itself included).  The pages print this window two ways
  *    ("[i-W, i-1]" and "j = i-W .. i"); the reading above is the one under
