@@ -186,6 +186,23 @@ def barrier(world: int):
         dist.barrier()
 
 
+def bench_config(hp, world: int) -> dict:
+    """The workload description both arms print (native and reference)."""
+    return {
+        "workload": hp.name,
+        "B": hp.B, "N": hp.N, "W": hp.W, "Hq": hp.Hq, "Hkv": hp.Hkv, "D": hp.D,
+        "parallelism": f"replicas{world}" if world > 1 else "single",
+        "l2": "inputs larger than L2 (prefill q/k/v/out 640 MB, decode cache 1 GB); no flush",
+        "step": "one-shot prefill + 4-chunk prefill (N=16384) + 128 decode steps (B=64, graph)",
+    }
+
+
+# nominal B200 figures (datasheet, dense): fractions against them are reported
+# beside the ones against the measured peaks, which are the roofline
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 # ---------------------------------------------------------------- CPU oracle sample
 
 _ORACLE_CACHE = {}
@@ -432,13 +449,7 @@ def run_native(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
-            "config": {
-                "workload": hp.name,
-                "B": hp.B, "N": hp.N, "W": hp.W, "Hq": hp.Hq, "Hkv": hp.Hkv, "D": hp.D,
-                "parallelism": f"replicas{world}" if world > 1 else "single",
-                "l2": "inputs larger than L2 (prefill q/k/v/out 640 MB, decode cache 1 GB); no flush",
-                "step": "one-shot prefill + 4-chunk prefill (N=16384) + 128 decode steps (B=64, graph)",
-            },
+            "config": bench_config(hp, world),
             "roofline": {
                 "bound": "hbm",
                 "kernel": "swa_decode (swa_decode_kernel<128,4> + swa_decode_combine_kernel<128,4>)",
@@ -448,6 +459,8 @@ def run_native(args):
                 "unit": "GB/s",
                 "frac": dec_call_gbs / peaks["hbm_gbs"],
                 "peak_kind": f"HBM copy ({peaks['source']})",
+                "frac_nominal": dec_call_gbs / NOMINAL_HBM_GBS,
+                "nominal_peak": NOMINAL_HBM_GBS,
                 "traffic": ncu_traffic("swa_decode_kernel<128,4>"),
                 "algorithmic_bytes_per_launch": dec_call_bytes / dw.steps,
                 "avg_launch_us": dec_call_ms * 1e3 / dw.steps,
@@ -461,6 +474,8 @@ def run_native(args):
                 "frac": achieved / peaks["bf16"],
                 "peak_kind": f"bf16 dense burst ({peaks['source']})",
                 "frac_of_sustained": achieved / peaks["bf16_sustained"],
+                "frac_nominal": achieved / NOMINAL_BF16_TFLOPS,
+                "nominal_peak": NOMINAL_BF16_TFLOPS,
                 "traffic": traffic,
                 "algorithmic_flops_per_launch": pf_flops,
             },
@@ -518,25 +533,21 @@ def _time_ms(fn, iters: int) -> float:
 def measure_sweep(swa, wl, dev, iters, world):
     """The long-prefill sweep (B=2, 32/8 heads, D=128): N in {4K, 8K, 16K, 32K}
     x W in {1024, 4096}, plus the dense-causal control W = N; useful TFLOP/s
-    and ms per launch (CUDA events, median).  Inputs are drawn on the device
-    (N(0,1) bf16, 1% of key rows x8), for timing only: the same shapes are
-    checked against the oracle in the tests.  Also the time ratio of dense
-    causal to W=4096 at N=16K, the pages' "about 2x faster at 16K" setting."""
+    and ms per launch (CUDA events, median).  The inputs are the seeded
+    ``workloads.sweep_point`` draws (1% of key rows x8), the same tensors the
+    parity tests compare with the oracle at every point.  Also the time ratio
+    of dense causal to W=4096 at N=16K, the pages' "about 2x faster at 16K"
+    setting."""
     import torch
-    B, Hq, Hkv, D = 2, 32, 8, 128
-    scale = 1.0 / D ** 0.5
-    g = torch.Generator(device=dev)
     res = {}
-    for N in (4096, 8192, 16384, 32768):
-        g.manual_seed(2000 + N)
-        q = torch.randn(B, N, Hq, D, device=dev, generator=g).to(torch.bfloat16)
-        k = torch.randn(B, N, Hkv, D, device=dev, generator=g)
-        k = (k * torch.where(torch.rand(B, N, Hkv, 1, device=dev, generator=g) < 0.01, 8.0, 1.0)).to(torch.bfloat16)
-        v = torch.randn(B, N, Hkv, D, device=dev, generator=g).to(torch.bfloat16)
+    for N in wl.SWEEP_N:
+        w0 = wl.sweep_point(N, 4096)
+        q, k, v = (t.to(dev) for t in wl.prefill_inputs(w0))
         out = torch.empty_like(q)
-        for W in sorted({1024, 4096, N}):
-            ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill(q, k, v, W, scale, out=out), iters), world)
-            tf = wl.useful_flops(B, N, W, Hq, D) / (ms * 1e-3) / 1e12
+        for W in sorted(set(wl.SWEEP_W) | {N}):
+            w = wl.sweep_point(N, W)
+            ms = max_over_ranks(_time_ms(lambda: swa.swa_prefill(q, k, v, w.W, w.scale, out=out), iters), world)
+            tf = wl.useful_flops(w.B, N, W, w.Hq, w.D) / (ms * 1e-3) / 1e12
             res[f"N{N}_W{W}" + ("_dense" if W == N else "")] = {"tflops": tf, "ms": ms}
         del q, k, v, out
     res["dense_over_swa_time_N16384_W4096"] = res["N16384_W16384_dense"]["ms"] / res["N16384_W4096"]["ms"]
@@ -657,8 +668,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": hp.name, "B": hp.B, "N": hp.N, "W": hp.W, "Hq": hp.Hq,
-                   "Hkv": hp.Hkv, "D": hp.D},
+        "config": bench_config(hp, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

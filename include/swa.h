@@ -167,7 +167,9 @@ size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W);
  *    before anything is launched (B=64, Hq=32, D=128, W=4096 needs 8.5 MB);
  *  - the first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture;
+ *    before any stream capture.  The address is kept for the life of the
+ *    process: resetting the device (cudaDeviceReset) after that first call is
+ *    not supported, since the kept address would no longer be valid;
  *  - all calls share the one array and it keeps the last call's contents;
  *    nothing in it needs to start at zero.  Calls that overlap on the GPU
  *    (different streams, or different host threads without ordering) race on

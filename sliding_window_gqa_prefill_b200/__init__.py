@@ -239,7 +239,7 @@ def swa_decode(q, k_cache, v_cache, pos, scale: float, out=None, workspace=None,
     need = swa_decode_workspace_size(B, Hq, Hkv, D, W)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    head = (_bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+    head = (_bf16(q, "q"), _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
             _i32(pos, "pos", B), _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale))
     tail = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rope_theta is None:
@@ -257,8 +257,8 @@ def swa_decode_noalloc(q, k_cache, v_cache, pos, scale: float, out, stream=None)
     B, Hq, D = q.shape
     W, Hkv = k_cache.shape[1], k_cache.shape[2]
     _check(lib().swa_decode_noalloc(
-        _bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)), _i32(pos, "pos", B),
-        _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale), _stream_handle(stream)),
+        _bf16(q, "q"), _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _i32(pos, "pos", B), _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, float(scale), _stream_handle(stream)),
         "swa_decode_noalloc")
     return out
 
@@ -378,7 +378,7 @@ def swa_decode_sinks(q, k_cache, v_cache, k_sink, v_sink, pos, scale: float, out
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check(lib().swa_decode_sinks(
-        _bf16(q, "q"), _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
+        _bf16(q, "q"), _bf16(k_cache, "k_cache", (B, W, Hkv, D)), _bf16(v_cache, "v_cache", (B, W, Hkv, D)),
         _bf16(k_sink, "k_sink", (B, S, Hkv, D)), _bf16(v_sink, "v_sink", (B, S, Hkv, D)), _i32(pos, "pos", B),
         _bf16(out, "out", (B, Hq, D)), B, Hq, Hkv, D, W, S, float(scale), workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream_handle(stream)), "swa_decode_sinks")

@@ -85,6 +85,9 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
     assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
     assert d["config"]["workload"] and d["vs_baseline"] is None
+    # the same workload description as the native arm's line
+    from sliding_window_gqa_prefill_b200 import workloads as wl
+    assert d["config"] == bench.bench_config(wl.HEADLINE_PREFILL, 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] == 4 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

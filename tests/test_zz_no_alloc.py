@@ -55,6 +55,9 @@ def test_noalloc_decode_matches_workspace_decode_twice():
                                   out_new.data_ptr(), B, Hq, Hkv, D, W, scale, stream)
         assert st == swa.SWA_OK, f"call {call}: status {st}"
         torch.cuda.synchronize()
+        # the same kernels on the same inputs: the same bits, whatever the
+        # previous call left in the shared scratch
+        assert torch.equal(out_new, out_ref), f"call {call}: differs from swa_decode"
         a = out_new.float().cpu().numpy()
         b = out_ref.float().cpu().numpy()
         assert np.isfinite(a).all(), f"call {call}: non-finite output"
