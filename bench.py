@@ -45,7 +45,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--ncu-case", choices=["prefill", "prefill_b2", "chunk", "decode"], default=None,
                     help="run a reduced case of one kernel three times for an ncu capture (no timing)")
     return ap.parse_args(argv)
 
@@ -686,14 +686,33 @@ def run_ncu_case(case: str) -> None:
     import sliding_window_gqa_prefill_b200 as swa
     from sliding_window_gqa_prefill_b200 import workloads as wl
     swa.lib()
-    if case == "prefill":
-        w = dataclasses.replace(wl.HEADLINE_PREFILL, B=1)
+    if case in ("prefill", "prefill_b2"):
+        w = wl.HEADLINE_PREFILL if case == "prefill_b2" else dataclasses.replace(wl.HEADLINE_PREFILL, B=1)
         q, k, v = (t.cuda() for t in wl.prefill_inputs(w))
         for _ in range(3):
             swa.swa_prefill(q, k, v, w.W, w.scale)
         alg = (q.numel() + k.numel() + v.numel() + q.numel()) * 2
-        print(f"ncu case prefill {w.name} B=1: algorithmic bytes per launch {alg}, "
+        print(f"ncu case {case} {w.name} B={w.B}: algorithmic bytes per launch {alg}, "
               f"useful FLOPs {wl.useful_flops(w.B, w.N, w.W, w.Hq, w.D)}")
+    elif case == "chunk":
+        # the benchmark's chunked prefill as it runs (B=1, 4 chunks of 4096
+        # through a 4096-slot buffer): per chunk one attention launch, then the
+        # append launch of 4096 rows; the 4th chunk reads a full buffer
+        w = wl.CHUNKED_16K
+        q, k, v = (t.cuda() for t in wl.chunked_inputs(w))
+        kc = torch.zeros(w.B, w.W, w.Hkv, w.D, dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        for s0 in range(0, w.N, w.C):
+            st = torch.full((w.B,), s0, dtype=torch.int32, device="cuda")
+            swa.swa_prefill_chunk(q[:, s0:s0 + w.C].contiguous(), k[:, s0:s0 + w.C].contiguous(),
+                                  v[:, s0:s0 + w.C].contiguous(), kc, vc, st, w.W, w.scale)
+        rows = w.B * w.C
+        alg_attn = rows * (w.Hq * 2 + w.Hkv * 2 * 2) * w.D * 2 + 2 * w.B * w.W * w.Hkv * w.D * 2
+        alg_append = 2 * 2 * rows * w.Hkv * w.D * 2
+        print(f"ncu case chunk {w.name}: 4th chunk attention algorithmic bytes {alg_attn} (q, k, v, out of "
+              f"the chunk + full K/V buffer), useful FLOPs "
+              f"{wl.useful_flops(w.B, w.N, w.W, w.Hq, w.D) - wl.useful_flops(w.B, w.N - w.C, w.W, w.Hq, w.D)}; "
+              f"append of {w.C} rows algorithmic bytes {alg_append} (k, v read and written)")
     else:
         w = dataclasses.replace(wl.DECODE_B64, B=16, steps=1)
         d = wl.decode_inputs(w)

@@ -10,6 +10,7 @@ streams.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -22,12 +23,15 @@ __all__ = [
     "swa_decode_sinks", "swa_rope", "swa_get_device_status", "swa_set_wait_limit_ns",
     "swa_selftest_wait_timeout", "swa_selftest_exp2", "SWA_OK", "SWA_ERR_INVALID_ARG",
     "SWA_ERR_UNSUPPORTED", "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_WINDOW_EXCL_LEFT",
-    "SWA_WINDOW_INCL_LEFT",
+    "SWA_WINDOW_INCL_LEFT", "bounds_checked",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_PKG)
 LIB_PATH = os.path.join(_PKG, "libswa.so")
+# the same library with every kernel index checked (SWA_BOUNDS_CHECK): a failed
+# check records SWA_ERR_INVALID_ARG and skips the access; for tests and debugging
+DEBUG_LIB_PATH = os.path.join(_PKG, "libswa_debug.so")
 HEADER = os.path.join(_ROOT, "include", "swa.h")
 _SOURCES = [os.path.join(_PKG, "csrc", f) for f in
             ("swa_api.cu", "device_common.cuh", "prefill_kernel.cuh", "decode_kernel.cuh")]
@@ -45,37 +49,56 @@ class SwaError(RuntimeError):
         name = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED", 3: "SWA_ERR_CUDA",
                 4: "SWA_ERR_TIMEOUT"}.get(status, f"status {status}")
         extra = ""
-        if status == SWA_ERR_CUDA and _lib is not None:
-            extra = f" (cuda error {_lib.swa_last_cuda_error()})"
+        if status == SWA_ERR_CUDA and _libs:
+            extra = f" (cuda error {lib().swa_last_cuda_error()})"
         super().__init__(f"{what}: {name}{extra}")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libswa.so for sm_100a in the package directory (nvcc)."""
-    stale = not os.path.exists(LIB_PATH) or any(
-        os.path.getmtime(s) > os.path.getmtime(LIB_PATH) for s in _SOURCES + [HEADER])
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile libswa.so (debug: libswa_debug.so, index-checked) for sm_100a in
+    the package directory (nvcc)."""
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    stale = not os.path.exists(path) or any(
+        os.path.getmtime(s) > os.path.getmtime(path) for s in _SOURCES + [HEADER])
     if force or stale:
-        tmp = LIB_PATH + f".tmp{os.getpid()}"
-        cmd = ["nvcc", *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []),
-               "-o", tmp, os.path.join(_PKG, "csrc", "swa_api.cu")]
+        tmp = path + f".tmp{os.getpid()}"
+        cmd = ["nvcc", *NVCC_FLAGS, *(["-DSWA_BOUNDS_CHECK"] if debug else []),
+               *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, os.path.join(_PKG, "csrc", "swa_api.cu")]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+        os.replace(tmp, path)
+    return path
 
 
 _lock = threading.Lock()
-_lib = None
+_libs = {}
+_use_debug = False
+
+
+@contextlib.contextmanager
+def bounds_checked():
+    """Within the block, every call goes to libswa_debug.so, whose kernels check
+    each row, slot and TMA coordinate they compute against its tensor's extent
+    (a failed check records SWA_ERR_INVALID_ARG; nothing traps).  Not
+    thread-safe: it switches the module-wide library."""
+    global _use_debug
+    prev = _use_debug
+    _use_debug = True
+    try:
+        yield
+    finally:
+        _use_debug = prev
 
 
 def lib() -> ctypes.CDLL:
-    """The loaded libswa.so.  Raises if it has not been built."""
-    global _lib
+    """The loaded libswa.so (libswa_debug.so inside bounds_checked()).  Raises
+    if it has not been built."""
+    path = DEBUG_LIB_PATH if _use_debug else LIB_PATH
     with _lock:
-        if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(f"libswa.so not built ({LIB_PATH}); call "
+        if path not in _libs:
+            if not os.path.exists(path):
+                raise RuntimeError(f"{os.path.basename(path)} not built ({path}); call "
                                    "sliding_window_gqa_prefill_b200.build()")
-            L = ctypes.CDLL(LIB_PATH)
+            L = ctypes.CDLL(path)
             vp, i, f, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
             L.swa_prefill.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, st]
             L.swa_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, st]
@@ -116,8 +139,8 @@ def lib() -> ctypes.CDLL:
                        L.swa_get_device_status, L.swa_set_wait_limit_ns,
                        L.swa_selftest_wait_timeout, L.swa_last_cuda_error):
                 fn.restype = ctypes.c_int
-            _lib = L
-    return _lib
+            _libs[path] = L
+    return _libs[path]
 
 
 def _check(status: int, what: str) -> None:

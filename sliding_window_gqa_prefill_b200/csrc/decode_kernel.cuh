@@ -10,20 +10,23 @@
 // GQA group read each K/V row once (section 3.4 of the manon006 review: GQA
 // cuts decode's cache reads).
 //
-// Memory-bound design (CUDA cores; the contraction is 4 x D per key, far
-// below what tensor cores need to pay off):
+// Memory-bound design: the kernel must stream the window's K and V rows at
+// HBM speed, so the arithmetic per key row has to stay a few instructions.
 //  * grid (split, kv head, sequence); a block of 4 warps streams one split of
-//    up to SPLIT keys.  Each lane owns 8 consecutive d of a key row, so a
-//    key row is read by D/8 lanes with 16-byte coalesced copies.
-//  * cp.async 16-byte copies into a per-warp 4-stage shared-memory ring keep
-//    several KB per warp in flight.
-//  * per key: partial dot products for all G heads of the group, reduced
-//    across the D/8 lanes of the row by a transposing butterfly (each level
-//    halves the values a lane holds), so a key x head score costs about one
-//    shuffle.  Online softmax per head in base 2 (scale folded into q); the
-//    exponent offset of a head is raised (exact maximum over the iteration,
+//    up to SPLIT keys in blocks of 16 keys, warp w taking blocks w, w+4, ...
+//  * each warp keeps its own 3-deep ring of 16-key K and V blocks in shared
+//    memory, filled by 16-byte cp.async copies (rows XOR-swizzled in 16-byte
+//    chunks so the matrix loads below are free of bank conflicts).
+//  * the G query heads of the group are the rows of a 16-row tensor-core
+//    tile (mma.sync m16n8k16, bf16 in, fp32 out; rows G..15 are zero):
+//    S = Q K^T for 16 keys is 2 x D/16 MMAs with K fed by ldmatrix, and
+//    O += P V is D/8 MMAs with V fed by ldmatrix.trans.  The S accumulator
+//    of a thread is exactly its A fragment of P (head = row, keys = columns),
+//    so P never leaves registers.  About 4 warp instructions per key row.
+//  * online softmax per head in base 2, scale applied to S in fp32; the
+//    exponent offset of a head is raised (exact maximum over the block,
 //    rescale of l and o) only when a score exceeds it by more than 2^8, so
-//    most iterations skip the per-iteration maximum entirely.
+//    most blocks take no maximum.
 //  * warps and splits are merged by log-sum-exp: in shared memory inside a
 //    block, and by swa_decode_combine_kernel across splits.
 #pragma once
@@ -34,27 +37,26 @@ namespace swa {
 
 constexpr int kDecodeSplit = 512;      // keys per block
 constexpr int kDecodeWarps = 4;
-constexpr int kDecodeStages = 4;
-
-__host__ __device__ constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x >> 1); }
+constexpr int kDecodeBlk = 16;         // keys per tensor-core block
+constexpr int kDecodeStages = 3;       // per-warp ring depth, in 16-key blocks
 
 template <int D, int G>
 struct DecodeCfg {
-    static constexpr int LPR = D / 8;                 // lanes per key row
-    static constexpr int R = 32 / LPR;                // key rows per warp-wide load
-    static constexpr int KPR = 4;                     // keys per row group per iteration
-    static constexpr int KI = R * KPR;                // keys per warp iteration
-    static constexpr int NV = KPR * G;                // partial sums per lane
-    static constexpr int TLEV = (ilog2c(NV) < ilog2c(LPR)) ? ilog2c(NV) : ilog2c(LPR);
-    static constexpr int VPL = NV >> TLEV;            // values per lane after the butterfly
-    static constexpr int STAGE_BYTES = 2 * KI * D * 2;   // K and V rows of one iteration
+    static constexpr int CH = D / 8;                       // 16-byte chunks per key row
+    static constexpr int ROW_BYTES = D * 2;
+    static constexpr int BLK_BYTES = kDecodeBlk * ROW_BYTES;   // K (or V) rows of one block
+    static constexpr int STAGE_BYTES = 2 * BLK_BYTES;          // K then V
     static constexpr int WARP_RING = kDecodeStages * STAGE_BYTES;
-    static constexpr int OFF_SCORE = kDecodeWarps * WARP_RING;   // per warp [KI][G] floats
-    static constexpr int OFF_MERGE = OFF_SCORE + kDecodeWarps * KI * G * 4;
+    static constexpr int RING_BYTES = kDecodeWarps * WARP_RING;
+    static constexpr int CPL = kDecodeBlk * CH / 32;           // 16-byte copies per lane, K or V
+    static constexpr int KSTEPS = D / 16;                      // MMA k-steps of S = Q K^T
+    static constexpr int NB = D / 8;                           // 8-column blocks of O
+    // the warp merge reuses the rings once every copy has landed
     static constexpr int MERGE_BYTES = kDecodeWarps * G * (D + 2) * 4;
-    static constexpr int SMEM_BYTES = OFF_MERGE + MERGE_BYTES;
+    static constexpr int SMEM_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "group size 1, 2, 4 or 8");
+    static_assert(CPL * 32 == kDecodeBlk * CH, "copies per lane");
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -66,34 +68,40 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// G consecutive floats of shared memory, vectorised where G allows.
-template <int G>
-__device__ __forceinline__ void load_g(const float *p, float (&out)[G]) {
-    if constexpr (G % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < G / 4; ++i) {
-            const float4 t = reinterpret_cast<const float4 *>(p)[i];
-            out[4 * i] = t.x;
-            out[4 * i + 1] = t.y;
-            out[4 * i + 2] = t.z;
-            out[4 * i + 3] = t.w;
-        }
-    } else if constexpr (G == 2) {
-        const float2 t = *reinterpret_cast<const float2 *>(p);
-        out[0] = t.x;
-        out[1] = t.y;
-    } else {
-        out[0] = p[0];
-    }
+// Four 8x8 bf16 matrices from shared memory (each lane gives one row address:
+// lanes 8i..8i+7 the rows of matrix i); register i of a lane holds two
+// adjacent elements of row lane/4 of matrix i (transposed: of column lane/4).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+// D(16x8, fp32) += A(16x16, bf16) B(16x8, bf16), warp-wide.  Only rows 0..7
+// of A are given (a0: columns 2t, 2t+1 and a2: columns 2t+8, 2t+9 of row
+// lane/4, t = lane%4); rows 8..15 are zero, so only d0 = D[lane/4][2t] and
+// d1 = D[lane/4][2t+1] are accumulated and returned.
+__device__ __forceinline__ void mma_rows8(float &d0, float &d1, uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+    [[maybe_unused]] float u2, u3;     // rows 8..15 of D: zero, not kept
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d0), "=f"(d1), "=f"(u2), "=f"(u3)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0), "f"(d1), "f"(0.f), "f"(0.f));
+}
+
+// Shared-memory offset of 16-byte chunk `ch` of row `r` in a block of rows of
+// `row_bytes`: chunks XOR-swizzled by the row's low three bits, so the eight
+// rows of one 8x8 matrix load fall in eight different bank groups.
+__device__ __forceinline__ uint32_t swz_off(int r, int ch, int row_bytes) {
+    return (uint32_t)(r * row_bytes + ((ch ^ (r & 7)) << 4));
 }
 
 // Partial result of one (sequence, kv head, split): per head m (base-2 max),
@@ -102,7 +110,7 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
 // SINKS: keys past the window's come from the sink buffer (attention sinks);
 // compiled out of the plain decode.
 template <int D, int G, bool SINKS>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 2)
 swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kc,
                   const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ pos,
                   __nv_bfloat16 *__restrict__ out, float2 *__restrict__ ws_ml,
@@ -110,8 +118,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                   int rope, const RopeTable rope_freq, const __nv_bfloat16 *__restrict__ ksink,
                   const __nv_bfloat16 *__restrict__ vsink, int S) {
     using Cfg = DecodeCfg<D, G>;
-    constexpr int LPR = Cfg::LPR, KPR = Cfg::KPR, KI = Cfg::KI, NV = Cfg::NV;
-    constexpr int TLEV = Cfg::TLEV, VPL = Cfg::VPL;
+    constexpr int CH = Cfg::CH, RB = Cfg::ROW_BYTES;
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -132,264 +139,169 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = lane / LPR;             // row group of this lane
-    const int sub = lane % LPR;             // which 8 d of the row
-    const uint32_t ring = smem_addr(smem + warp * Cfg::WARP_RING);
-    float *score = reinterpret_cast<float *>(smem + Cfg::OFF_SCORE) + warp * KI * G;
+    const int hr = lane >> 2;                // fragment row: head of the group (valid if < G)
+    const int t4 = lane & 3;                 // fragment column pair
+    const bool head_ok = hr < G;
+    const uint32_t ring = smem_addr(smem) + warp * Cfg::WARP_RING;
 
-    // q for every head of the group, d = sub*8 .. sub*8+7, pre-scaled to base 2,
-    // as four (even, odd) pairs for the packed two-lane FMA
-    float2 q2[G][4];
+    // A fragments of Q (row hr; columns kk*16 + 2*t4 + {0, 1} and + 8), bf16;
+    // with rope, each pair (2i, 2i+1) rotated at position p in fp32 first
+    uint32_t qa[Cfg::KSTEPS][2];
+    {
+        const __nv_bfloat16 *qrow = q + ((size_t)b * Hq + g * G + (head_ok ? hr : 0)) * D;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)b * Hq + g * G + h) * D) + sub);
-        float qf[8];
-        bf16x8_to_f32(raw, qf);
-        if (rope) {            // rotary embedding of the query at its position, in fp32
+        for (int kk = 0; kk < Cfg::KSTEPS; ++kk)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float c, sn;
-                rope_cos_sin((double)p, rope_freq.f[sub * 4 + e], c, sn);
-                const float x0 = qf[2 * e], x1 = qf[2 * e + 1];
-                qf[2 * e] = x0 * c - x1 * sn;
-                qf[2 * e + 1] = x0 * sn + x1 * c;
+            for (int hf = 0; hf < 2; ++hf) {
+                const int d = kk * 16 + hf * 8 + 2 * t4;
+                uint32_t w = head_ok ? __ldg(reinterpret_cast<const uint32_t *>(qrow + d)) : 0u;
+                if (rope && head_ok) {
+                    float c, sn;
+                    rope_cos_sin((double)p, rope_freq.f[d >> 1], c, sn);
+                    const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
+                    w = pack_bf16x2(x0 * c - x1 * sn, x0 * sn + x1 * c);
+                }
+                qa[kk][hf] = w;
             }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) q2[h][e] = make_float2(qf[2 * e] * scale_log2, qf[2 * e + 1] * scale_log2);
     }
 
     const size_t row_stride = (size_t)Hkv * D;     // elements between consecutive slots
-    const __nv_bfloat16 *kbase = kc + ((size_t)b * W * Hkv + g) * D + sub * 8;
-    const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv + g) * D + sub * 8;
-    const __nv_bfloat16 *ksbase = ns ? ksink + ((size_t)b * S * Hkv + g) * D + sub * 8 : kbase;
-    const __nv_bfloat16 *vsbase = ns ? vsink + ((size_t)b * S * Hkv + g) * D + sub * 8 : vbase;
+    const __nv_bfloat16 *kbase = kc + ((size_t)b * W * Hkv + g) * D;
+    const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv + g) * D;
+    const __nv_bfloat16 *ksbase = ns ? ksink + ((size_t)b * S * Hkv + g) * D : kbase;
+    const __nv_bfloat16 *vsbase = ns ? vsink + ((size_t)b * S * Hkv + g) * D : vbase;
 
-    const int n_iter_total = (end - begin + KI - 1) / KI;
-    const int my_iters = (n_iter_total > warp) ? (n_iter_total - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+    const int nblk = (end - begin + kDecodeBlk - 1) / kDecodeBlk;
+    const int my_blocks = (nblk > warp) ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
 
-    // stage layout: K rows [KI][D] then V rows [KI][D]
-    auto issue = [&](int it_local, int stage) {
-        const int it = warp + it_local * kDecodeWarps;
+    // stage layout: K rows [16][D] then V rows [16][D], swizzled chunks
+    auto issue = [&](int i_local, int stage) {
+        const int blk = warp + i_local * kDecodeWarps;
         const uint32_t st = ring + stage * Cfg::STAGE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < KPR; ++kk) {
-            const int kr = row * KPR + kk;
-            const int key = min(begin + it * KI + kr, end - 1);      // clamp: always in bounds
-            const uint32_t off = (uint32_t)((kr * D + sub * 8) * 2);
-            if (SINKS) {
-                const bool sink = key >= Lw;
-                const size_t rowi = (size_t)(sink ? key - Lw : key) * row_stride;
-                cp_async16(st + off, (sink ? ksbase : kbase) + rowi);
-                cp_async16(st + KI * D * 2 + off, (sink ? vsbase : vbase) + rowi);
+        for (int c = 0; c < Cfg::CPL; ++c) {
+            const int id = c * 32 + lane;
+            const int r = id / CH, ch = id % CH;
+            const int key = min(begin + blk * kDecodeBlk + r, end - 1);     // clamp: always in bounds
+            const uint32_t off = swz_off(r, ch, RB);
+            if (SINKS && key >= Lw) {
+                if (!in_bounds(key - Lw, S)) continue;
+                const size_t rowi = (size_t)(key - Lw) * row_stride + ch * 8;
+                cp_async16(st + off, ksbase + rowi);
+                cp_async16(st + Cfg::BLK_BYTES + off, vsbase + rowi);
             } else {
-                cp_async16(st + off, kbase + (size_t)key * row_stride);
-                cp_async16(st + KI * D * 2 + off, vbase + (size_t)key * row_stride);
+                if (!in_bounds(key, W)) continue;
+                const size_t rowi = (size_t)key * row_stride + ch * 8;
+                cp_async16(st + off, kbase + rowi);
+                cp_async16(st + Cfg::BLK_BYTES + off, vbase + rowi);
             }
         }
     };
 
-    // m_run: running base-2 maximum per head (equal in all lanes);
-    // l_run: this lane's share of the running sum per head (each key x head
-    // is counted by exactly one lane); o2: this lane's row-group partial of
-    // the output for its 8 d, per head
-    float m_run[G], l_run[G];
-    float2 o2[G][4];
+    // per thread: head hr's running offset (equal in the 4 lanes of a quad),
+    // this lane's share of its sum, and O[hr][nb*8 + 2*t4 + {0, 1}]
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[Cfg::NB][2];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        m_run[h] = -INFINITY;
-        l_run[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o2[h][e] = make_float2(0.f, 0.f);
-    }
+    for (int nb = 0; nb < Cfg::NB; ++nb) o[nb][0] = o[nb][1] = 0.f;
 
 #pragma unroll
     for (int s = 0; s < kDecodeStages - 1; ++s) {
-        if (s < my_iters) issue(s, s);
+        if (s < my_blocks) issue(s, s);
         cp_async_commit();
     }
 
-    // value index of v[i] after the butterfly = vidx0 + i; lanes that only
-    // hold copies (when NV < LPR) do not write
-    int vidx0 = 0;
-    {
-        int half = NV;
-#pragma unroll
-        for (int lev = 0; lev < TLEV; ++lev) {
-            half >>= 1;
-            const int off = LPR >> (lev + 1);
-            if (sub & off) vidx0 += half;
-        }
-    }
-    const bool writer = (TLEV == ilog2c(LPR)) || ((sub & ((LPR >> TLEV) - 1)) == 0);
-
-    for (int it_local = 0; it_local < my_iters; ++it_local) {
-        const int stage = it_local % kDecodeStages;
+    for (int i = 0; i < my_blocks; ++i) {
+        const int stage = i % kDecodeStages;
         cp_async_wait<kDecodeStages - 2>();
         __syncwarp();
         {
-            const int nxt = it_local + kDecodeStages - 1;
-            if (nxt < my_iters) issue(nxt, nxt % kDecodeStages);
+            const int nxt = i + kDecodeStages - 1;
+            if (nxt < my_blocks) issue(nxt, nxt % kDecodeStages);
             cp_async_commit();
         }
-        const uint8_t *st = smem + warp * Cfg::WARP_RING + stage * Cfg::STAGE_BYTES;
-        const int it = warp + it_local * kDecodeWarps;
-        const int key_base = begin + it * KI;
+        const uint32_t sk = ring + stage * Cfg::STAGE_BYTES, sv = sk + Cfg::BLK_BYTES;
+        const int key0 = begin + (warp + i * kDecodeWarps) * kDecodeBlk;
 
-        // partial dot products over this lane's 8 d: value index kk*G + h
-        float v[NV];
+        // S = Q K^T: keys 0-7 and 8-15 of the block; ldmatrix x4 covers 32 d
+        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int kk = 0; kk < KPR; ++kk) {
-            const int kr = row * KPR + kk;
-            float kf[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(st + (kr * D + sub * 8) * 2), kf);
+        for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc = ffma2(q2[h][e], make_float2(kf[2 * e], kf[2 * e + 1]), acc);
-                v[kk * G + h] = acc.x + acc.y;
+            for (int c4 = 0; c4 < CH / 4; ++c4) {
+                const int r = nb * 8 + (lane & 7), ch = c4 * 4 + (lane >> 3);
+                uint32_t kb[4];
+                ldsm_x4(sk + swz_off(r, ch, RB), kb);
+                mma_rows8(s[nb][0], s[nb][1], qa[2 * c4][0], qa[2 * c4][1], kb[0], kb[1]);
+                mma_rows8(s[nb][0], s[nb][1], qa[2 * c4 + 1][0], qa[2 * c4 + 1][1], kb[2], kb[3]);
             }
+        // this lane's scores of head hr: keys key0 + 2*t4 + {0, 1, 8, 9}
+        float sc[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int key = key0 + 2 * t4 + (e & 1) + (e >> 1) * 8;
+            sc[e] = (key < end) ? sc[e] * scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[e]);
         }
-        // transposing butterfly across the LPR lanes of the row
+        // a score more than 2^8 above its head's offset (always on the first
+        // block) makes the warp take the exact maximum over the block (the
+        // quad of lanes holding the head) and rescale; otherwise the offset
+        // stays (p = 2^(s - offset) <= 2^8, exact after normalisation)
+        if (__any_sync(0xffffffffu, head_ok && mx > m_run + 8.0f)) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            if (mx > m_run) {                    // uniform across the quad
+                const float alpha = ex2_approx(m_run - mx);      // 0 when m_run = -inf
+                l_run *= alpha;
 #pragma unroll
-        for (int lev = 0; lev < ilog2c(LPR); ++lev) {
-            const int off = LPR >> (lev + 1);
-            if (lev < TLEV) {
-                const int half = NV >> (lev + 1);
-                const bool upper = (sub & off) != 0;
-#pragma unroll
-                for (int i = 0; i < NV / 2; ++i) {
-                    if (i < half) {
-                        const float send = upper ? v[i] : v[i + half];
-                        const float keep = upper ? v[i + half] : v[i];
-                        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                    }
+                for (int nb = 0; nb < Cfg::NB; ++nb) {
+                    o[nb][0] *= alpha;
+                    o[nb][1] *= alpha;
                 }
-            } else {
-#pragma unroll
-                for (int i = 0; i < VPL; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
+                m_run = mx;
             }
         }
-        // keys past the split masked; a score more than 2^8 above the running
-        // offset of its head (always so on the first iteration) makes the warp
-        // take the exact maximum over the iteration and rescale; otherwise the
-        // offset stays (p = 2^(s - offset) <= 2^8, exact after normalisation)
-        bool big = false;
-        if (writer) {
+        float pw[4];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int idx = vidx0 + i;
-                const int kr = row * KPR + idx / G, h = idx % G;
-                v[i] = (key_base + kr < end) ? v[i] : -INFINITY;
-                float mh = m_run[0];
-#pragma unroll
-                for (int hh = 1; hh < G; ++hh) mh = (h == hh) ? m_run[hh] : mh;
-                big |= v[i] > mh + 8.0f;
-            }
+        for (int e = 0; e < 4; ++e) pw[e] = head_ok ? ex2_approx(sc[e] - m_run) : 0.f;
+        // P as the A fragment of O += P V: columns (keys) 2*t4 + {0, 1} and + 8;
+        // l sums P as rounded to bf16, the weights V is actually multiplied by
+        const uint32_t pa0 = pack_bf16x2(pw[0], pw[1]), pa2 = pack_bf16x2(pw[2], pw[3]);
+        {
+            const float2 l2 = add_bf16x2(add_bf16x2(make_float2(0.f, 0.f), pa0), pa2);
+            l_run += l2.x + l2.y;
         }
-        if (__any_sync(0xffffffffu, big)) {
-            if (writer) {
 #pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int idx = vidx0 + i;
-                    score[(row * KPR + idx / G) * G + idx % G] = v[i];
-                }
-            }
-            __syncwarp();
-            float m_new[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) m_new[h] = m_run[h];
-#pragma unroll
-            for (int kr = 0; kr < KI; ++kr) {
-                float sv[G];
-                load_g<G>(score + kr * G, sv);
-#pragma unroll
-                for (int h = 0; h < G; ++h) m_new[h] = fmaxf(m_new[h], sv[h]);
-            }
-            __syncwarp();                        // every lane has read the scores
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                if (m_new[h] > m_run[h]) {       // uniform across the warp
-                    const float alpha = ex2_approx(m_run[h] - m_new[h]);   // 0 when m_run = -inf
-                    l_run[h] *= alpha;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) o2[h][e] = make_float2(o2[h][e].x * alpha, o2[h][e].y * alpha);
-                    m_run[h] = m_new[h];
-                }
-            }
-        }
-        // one exponential per key x head, by the lane that holds it
-        if (writer) {
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int idx = vidx0 + i;
-                const int kr = row * KPR + idx / G, h = idx % G;
-                float mh = m_run[0];
-#pragma unroll
-                for (int hh = 1; hh < G; ++hh) mh = (h == hh) ? m_run[hh] : mh;
-                const float pw = ex2_approx(v[i] - mh);
-#pragma unroll
-                for (int hh = 0; hh < G; ++hh) l_run[hh] += (h == hh) ? pw : 0.f;
-                score[kr * G + h] = pw;
-            }
-        }
-        __syncwarp();
-        // P V for the KPR keys of this lane's row
-#pragma unroll
-        for (int kk = 0; kk < KPR; ++kk) {
-            const int kr = row * KPR + kk;
-            float vf[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(st + KI * D * 2 + (kr * D + sub * 8) * 2), vf);
-            float pw[G];
-            load_g<G>(score + kr * G, pw);
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float2 p2 = make_float2(pw[h], pw[h]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o2[h][e] = ffma2(p2, make_float2(vf[2 * e], vf[2 * e + 1]), o2[h][e]);
-            }
+        for (int c2 = 0; c2 < CH / 2; ++c2) {
+            const int mi = lane >> 3;
+            const int r = (mi & 1) * 8 + (lane & 7), ch = c2 * 2 + (mi >> 1);
+            uint32_t vb[4];
+            ldsm_x4_trans(sv + swz_off(r, ch, RB), vb);
+            mma_rows8(o[2 * c2][0], o[2 * c2][1], pa0, pa2, vb[0], vb[1]);
+            mma_rows8(o[2 * c2 + 1][0], o[2 * c2 + 1][1], pa0, pa2, vb[2], vb[3]);
         }
         __syncwarp();
     }
     cp_async_wait<0>();
 
-    // merge within the warp: o over the row groups (lanes with equal sub),
-    // l over every lane
+    // l over the quad (each lane summed its own keys)
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+
+    // merge the warps of the block in shared memory (over the rings)
+    __syncthreads();
+    float *mg = reinterpret_cast<float *>(smem);    // [warp][G][D+2]
+    if (head_ok) {
+        float *dst = mg + (warp * G + hr) * (D + 2);
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                o2[h][e].x += __shfl_xor_sync(0xffffffffu, o2[h][e].x, off);
-                o2[h][e].y += __shfl_xor_sync(0xffffffffu, o2[h][e].y, off);
-            }
-    }
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1)
-#pragma unroll
-        for (int h = 0; h < G; ++h) l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], off);
-    float o[G][8];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            o[h][2 * e] = o2[h][e].x;
-            o[h][2 * e + 1] = o2[h][e].y;
+        for (int nb = 0; nb < Cfg::NB; ++nb) {
+            dst[nb * 8 + 2 * t4] = o[nb][0];
+            dst[nb * 8 + 2 * t4 + 1] = o[nb][1];
         }
-    // merge the warps of the block in shared memory
-    float *mg = reinterpret_cast<float *>(smem + Cfg::OFF_MERGE);    // [warp][G][D+2]
-    if (row == 0) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float *dst = mg + (warp * G + h) * (D + 2);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dst[sub * 8 + e] = o[h][e];
-            if (sub == 0) {
-                dst[D] = m_run[h];
-                dst[D + 1] = l_run[h];
-            }
+        if (t4 == 0) {
+            dst[D] = m_run;
+            dst[D + 1] = l_run;
         }
     }
     __syncthreads();
@@ -407,9 +319,11 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             acc += src[d] * sc;
         }
         if (nsplit == 1) {
-            out[((size_t)b * Hq + g * G + h) * D + d] = __float2bfloat16_rn(acc / l);
+            const size_t oi = ((size_t)b * Hq + g * G + h) * D + d;
+            if (in_bounds((long long)oi, (long long)gridDim.z * Hq * D)) out[oi] = __float2bfloat16_rn(acc / l);
         } else {
             const size_t slot = ((size_t)(b * Hkv + g) * nsplit_max + split) * G + h;
+            if (!in_bounds(split, nsplit_max)) continue;
             ws_o[slot * D + d] = acc;
             if (d == 0) ws_ml[slot] = make_float2(m, l);
         }
@@ -429,7 +343,7 @@ swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restr
     const int ns = (S > 0 && p >= W) ? min(S, p - W + 1) : 0;
     const int L = ((p >= W - 1) ? W : p + 1) + ns;
     const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
-    if (nsplit <= 1) return;
+    if (nsplit <= 1 || !in_bounds(nsplit - 1, nsplit_max)) return;
     const size_t base = (size_t)(b * Hkv + g) * nsplit_max;
     constexpr int kUnrolled = 16;            // splits loaded side by side (W <= 8192)
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
@@ -496,13 +410,14 @@ __global__ void swa_append_kernel(const uint4 *__restrict__ k_new, const uint4 *
         }
         const long long p = (long long)p0 + t;
         const int slot = (int)(p % W);
+        if (!in_bounds(slot, W) || !in_bounds(b, B)) continue;
         const size_t dst = ((size_t)b * W + slot) * row_vec + c;
         uint4 kv = __ldg(k_new + i);
         if (rope) kv = rope_rotate8(kv, (c % head_vec) * 4, (double)p, rope_freq);
         const uint4 vv = __ldg(v_new + i);
         k_cache[dst] = kv;
         v_cache[dst] = vv;
-        if (p < S) {                     // attention sinks: positions below S kept for good
+        if (p < S && in_bounds(p, S)) {  // attention sinks: positions below S kept for good
             const size_t sdst = ((size_t)b * S + p) * row_vec + c;
             k_sink[sdst] = kv;
             v_sink[sdst] = vv;
@@ -536,13 +451,14 @@ __global__ void swa_append_varlen_kernel(const uint4 *__restrict__ k_new, const 
         }
         const int c0 = __ldg(cu + lo), c1 = __ldg(cu + lo + 1);
         const int s0 = __ldg(start_pos + lo);
-        if (r < c0 || r >= c1 || s0 < 0) {            // malformed offsets or position
+        if (r < c0 || r >= c1 || c0 < 0 || c1 > total || s0 < 0) {   // malformed offsets or position
             record_status(kStatusInvalid);
             continue;
         }
         const int t = r - c0;
         if (t < (c1 - c0) - W) continue;              // overwritten later in this call
         const int slot = (int)(((long long)s0 + t) % W);
+        if (!in_bounds(slot, W) || !in_bounds(lo, B)) continue;
         const size_t dst = ((size_t)lo * W + slot) * row_vec + c;
         k_cache[dst] = __ldg(k_new + i);
         v_cache[dst] = __ldg(v_new + i);

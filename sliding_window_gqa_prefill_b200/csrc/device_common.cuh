@@ -28,6 +28,27 @@ __device__ __forceinline__ void record_status(int code) {
     atomicCAS(&g_status, 0, code);
 }
 
+// Index checks of the bounds-checked build (compiled with SWA_BOUNDS_CHECK):
+// every global row, slot and TMA start coordinate a kernel computes is checked
+// against the extent of its tensor before use.  A failed check records
+// SWA_ERR_INVALID_ARG in the status word and the access is skipped (or, for a
+// TMA load whose barrier must still complete, redirected to coordinate 0); no
+// trap.  In the normal build the checks compile to nothing.
+#ifdef SWA_BOUNDS_CHECK
+constexpr bool kBoundsCheck = true;
+#else
+constexpr bool kBoundsCheck = false;
+#endif
+
+__device__ __forceinline__ bool in_bounds(long long idx, long long n) {
+    if (!kBoundsCheck || (idx >= 0 && idx < n)) return true;
+    record_status(kStatusInvalid);
+    return false;
+}
+
+// A TMA start coordinate: itself when inside [0, n), else 0 (recorded).
+__device__ __forceinline__ int checked_coord(int c, int n) { return in_bounds(c, n) ? c : 0; }
+
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -337,6 +358,19 @@ __device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t *w) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// acc.x += low bf16 half of w, acc.y += high half (each widened exactly to
+// fp32).  Lets a softmax sum the weights it actually multiplies V by, i.e. P
+// after its rounding to bf16, so that O / l is a convex combination of the
+// value rows: when one key dominates a row, its rounding cancels instead of
+// showing as a relative error of the whole output.
+__device__ __forceinline__ float2 add_bf16x2(float2 acc, uint32_t w) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(w));
+    return acc;
 }
 
 // Rotary embedding frequencies theta^(-2i/D), i < D/2, computed on the host

@@ -100,6 +100,7 @@ struct PrefillCfg {
     // which of the 16 column pairs of each 32-column chunk take the polynomial
     // exponential instead of ex2.approx (bits 3, 7, 11, 15: one pair in four)
     static constexpr uint32_t kEmuPairs = 0x8888u;
+    static_assert(kEmuPairs == (kEmuPairs & 0xFu) * 0x1111u, "the pattern repeats every four pairs");
     // PV in two halves of 64 keys: the first half starts while the softmax
     // still computes the second half of P
     static constexpr bool kSplitPV = true;
@@ -131,6 +132,14 @@ struct UnitPlan {
     size_t orow0;    // output row of query row 0 of this sequence
 };
 
+// Rows of sequence b of a packed batch: cu_seqlens[b+1] - cu_seqlens[b] when
+// 0 <= cu[b] <= cu[b+1] <= total rows, else 0 (a malformed sequence is
+// skipped, so no row outside the packed tensors is ever read or written).
+__device__ __forceinline__ int varlen_rows(const PrefillParams &p, int b) {
+    const int c0 = __ldg(p.cu_seqlens + b), c1 = __ldg(p.cu_seqlens + b + 1);
+    return (c0 >= 0 && c0 <= c1 && c1 <= p.Nq) ? c1 - c0 : 0;
+}
+
 // pre: shared-memory prefix sums of query blocks per sequence (varlen only).
 __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, const int *pre) {
     constexpr int BM = 128, BN = 128;
@@ -150,8 +159,8 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         P.b = lo;
         P.qb = qbi - pre[lo];
         const int c0 = __ldg(p.cu_seqlens + lo);
-        P.nq = max(0, __ldg(p.cu_seqlens + lo + 1) - c0);
-        P.row0 = c0;
+        P.nq = varlen_rows(p, lo);
+        P.row0 = P.nq > 0 ? c0 : 0;
         P.tb = 0;
         P.orow0 = (size_t)c0;
     } else {
@@ -358,9 +367,9 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             int acc = 0;
             for (int b = 0; b < p.B; ++b) {
                 pre[b] = acc;
-                const int n = __ldg(p.cu_seqlens + b + 1) - __ldg(p.cu_seqlens + b);
-                if (n < 0) record_status(kStatusInvalid);
-                acc += (max(n, 0) + 127) / 128;
+                const int n = varlen_rows(p, b);
+                if (n == 0 && __ldg(p.cu_seqlens + b + 1) != __ldg(p.cu_seqlens + b)) record_status(kStatusInvalid);
+                acc += (n + 127) / 128;
             }
             pre[p.B] = acc;
             *unit_count = acc * p.Hkv * p.npairs;
@@ -403,10 +412,12 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int nact = 1 + P.act1;
                 if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
                 mbar_arrive_expect_tx(bar_q_full, nact * TB);
+                const int qrow = checked_coord(P.row0 + P.q0, p.Nq);
+                const int qb = checked_coord(P.tb, p.cu_seqlens ? 1 : p.B);
                 for (int t = 0; t < nact; ++t) {
-                    const int h = P.h0 + t;
+                    const int h = checked_coord(P.h0 + t, p.Hq);
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, P.row0 + P.q0, P.tb);
+                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, qrow, qb);
                 }
                 ++q_cnt;
                 for (int j = 0; j < P.n; ++j) {
@@ -417,7 +428,12 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     if (!mbar_wait_bounded(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, limit)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar_k_full + 8 * ks, TB);
                     // cache tiles: [B, W] slots of sequence b; main tiles: rows of this sequence
-                    const int krow = T.cache ? T.row0 : P.row0 + T.row0, kb = T.cache ? P.b : P.tb;
+                    int krow = T.cache ? T.row0 : P.row0 + T.row0, kb = T.cache ? P.b : P.tb;
+                    if (kBoundsCheck) {
+                        krow = checked_coord(krow, T.cache == 2 ? p.sink_buf : T.cache ? p.W : p.Nk);
+                        kb = checked_coord(kb, (T.cache || !p.cu_seqlens) ? p.B : 1);
+                        (void)checked_coord(P.g, p.Hkv);
+                    }
                     for (int r = 0; r < NREG; ++r)
                         tma_load_4d(sK + ks * TB + r * RB, mk, bar_k_full + 8 * ks, r * 64, P.g, krow, kb);
                     ++k_cnt[ks];
@@ -648,8 +664,17 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int c = 8; c < BN; c += 8)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
-                const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                // chain e of the tree holds the columns c with c mod 8 == e, i.e. column
+                // pair (e / 2) of every group of four pairs; kEmuPairs repeats every
+                // four pairs, so each chain holds columns of one exponential only:
+                // the maximum over the polynomial columns and over the others
+                float mpoly = -INFINITY, mmufu = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if ((Cfg::kEmuPairs >> (e >> 1)) & 1u) mpoly = fmaxf(mpoly, mx[e]);
+                    else mmufu = fmaxf(mmufu, mx[e]);
+                }
+                const float mt = fmaxf(mpoly, mmufu);
                 const float m_tile = mt * sl2;
                 const float m_cand = fmaxf(m_use, m_tile);
                 if (j == 0) {
@@ -702,7 +727,14 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
                 const float2 asum = fadd2(a01, a23);
-                l += asum.x + asum.y;
+                // l must sum the weights V is multiplied by, i.e. P as rounded to
+                // bf16.  Only the largest P matters (when one key dominates a row its
+                // rounding would scale the whole output; the others' average out): it
+                // is recomputed exactly as its element computed it, by the same
+                // exponential, and its rounding added
+                const float xm = fmaf(mt, sl2, -mb);
+                const float pm = (mpoly >= mmufu) ? exp2_poly2(make_float2(xm, xm)).x : ex2_approx(xm);
+                l += asum.x + asum.y + (__bfloat162float(__float2bfloat16_rn(pm)) - pm);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -716,7 +748,10 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             ++oc;
             tc_fence_after();
             const int h = P.h0 + t;
-            const bool valid_row = i_rel < P.nq;
+            bool valid_row = i_rel < P.nq;
+            if (kBoundsCheck && valid_row)
+                valid_row = in_bounds((long long)P.orow0 + i_rel, p.cu_seqlens ? p.Nq : (long long)p.B * p.Nq) &&
+                            in_bounds(h, p.Hq);
             const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
             __nv_bfloat16 *orow = p.out + ((P.orow0 + i_rel) * p.Hq + h) * D;
 #pragma unroll

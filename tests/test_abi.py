@@ -41,6 +41,21 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, n)
 
 
+def test_index_checked_library_exports_the_same_symbols():
+    """libswa_debug.so (SWA_BOUNDS_CHECK) is the same ABI: it builds, loads
+    without a GPU and exports every declared symbol."""
+    swa.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", swa.DEBUG_LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(swa_\w+)$", out, re.M))
+    assert not [n for n in declared_symbols() if n not in exported]
+    with swa.bounds_checked():
+        L = swa.lib()
+    assert L is not swa.lib() and L._name == swa.DEBUG_LIB_PATH
+    assert L.swa_prefill(None, 0x1000, 0x1000, 0x1000, 1, 16, 4, 2, 128, 8, 0, 0.1, None) == \
+        swa.SWA_ERR_INVALID_ARG
+
+
 def test_null_and_bad_sizes_rejected_without_device(lib):
     null = None
     ok_ptr = 0x1000            # aligned, never dereferenced: checks fail first
