@@ -676,11 +676,14 @@ def run_reference(args):
 
 
 def run_ncu_case(case: str) -> None:
-    """Reduced launches for ncu captures, the benchmark's kernels on a fraction
-    of its workload that still exceeds L2: prefill B=1 (half the headline
-    prefill, same per-unit structure), decode B=16 (a quarter of the batch,
-    positions from the same distribution).  Prints the algorithmic bytes per
-    launch so a capture's DRAM traffic can be scaled to the full launch."""
+    """Launches for ncu captures, each repeated so a capture can skip warm-up
+    launches: `prefill_b2` the headline prefill at its benchmark size (671 MB
+    on the device), `prefill` half of it (B=1, same per-unit structure),
+    `chunk` the benchmark's chunked prefill (4 x attention + append), `decode`
+    a reduced decode (B=16, a quarter of the batch, positions from the same
+    distribution, still above L2).  Prints the algorithmic bytes per launch so
+    a capture's DRAM traffic can be compared with (or scaled to) the
+    benchmark's launch."""
     import dataclasses
     import torch
     import sliding_window_gqa_prefill_b200 as swa
