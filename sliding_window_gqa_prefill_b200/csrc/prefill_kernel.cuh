@@ -16,7 +16,7 @@
 //  * Only key tiles that intersect the band [q0-W+1, q0+127] are visited, so
 //    work is O(N*W).  Tiles strictly inside the band skip all masking.
 //  * Warp roles (12 warps): warp 0 issues TMA loads (Q once per unit, K and V
-//    through 3- and 2-deep rings); warp 1 issues tcgen05.mma from one thread;
+//    through 2-deep rings); warp 1 issues tcgen05.mma from one thread;
 //    warp 2 owns the tensor-memory allocation; warps 4-7 and 8-11 are the
 //    softmax warpgroups of query head 0 and 1 of the pair.
 //  * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 columns each.  The
@@ -25,7 +25,9 @@
 //  * Online softmax in fp32, base-2 exponent with the scale folded in.  The
 //    running maximum used as exponent offset is raised only when the tile
 //    maximum exceeds it by more than 8 (2^8 bound on P), so the O rescale
-//    round trip through tensor memory is rare.
+//    round trip through tensor memory is rare.  P is rounded to bf16 for the
+//    PV MMA; l adds, per tile, the rounding of the tile's largest P (as its
+//    element computed it), so a row dominated by one key keeps O / l exact.
 //  * Chunked pre-fill: the key tiles of a unit are the cache slot tiles that
 //    hold positions inside the window of the block (one or two runs of slots
 //    modulo W), then the chunk's own tiles.  Slot s holds position
@@ -202,7 +204,7 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
             P.s0 = 0;
         }
         // sink positions j <= i - W exist for some row i of the block
-        P.sink_tile = (p.sink_buf > 0 && P.s0 + P.q0 + BM - 1 >= p.W) ? (p.sink_buf + BN - 1) / BN : 0;
+        P.sink_tile = (p.sink_buf > 0 && (long long)P.s0 + P.q0 + BM - 1 >= p.W) ? (p.sink_buf + BN - 1) / BN : 0;
         P.qs = P.s0 % p.W;
         // oldest age any row of the block still needs: age < W - q0, age <= s0
         const int A = min(p.W - P.q0 - 1, P.s0);
@@ -603,7 +605,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     ok = false;
                     break;
                 }
-                rope_row_swizzled<D>(smem + Cfg::OFF_Q + t * TB, row, (double)(P.s0 + i_rel), p.rope_freq);
+                rope_row_swizzled<D>(smem + Cfg::OFF_Q + t * TB, row, (double)P.s0 + i_rel, p.rope_freq);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_q_rot + 8 * t);
@@ -634,7 +636,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (T.masked) {
                     if (T.cache == 2) {
                         // sink slot j holds position j: visible iff outside the window
-                        const int lim = P.s0 + i_rel - p.W;
+                        const long long lim = (long long)P.s0 + i_rel - p.W;   // 64-bit: rows past the chunk too
 #pragma unroll
                         for (int c = 0; c < BN; ++c) {
                             const int slot = T.row0 + c;
