@@ -421,7 +421,10 @@ def run_native(args):
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = hout.numel() * 2
 
-    launches_per_step = 1 + len(c_chunks) * 2 + dw.steps * (2 + (1 if ws_bytes and dw.W > 512 else 0))
+    # per step: the one-shot prefill, attention + append per chunk, and per
+    # decode step the append, the split-KV kernel and the split merge (the
+    # window of 4096 keys spans several 1024-key splits, so the merge runs)
+    launches_per_step = 1 + len(c_chunks) * 2 + dw.steps * 3
 
     # ---- the widened rows, timed on their own (CUDA events, after the step)
     extras = measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, max(3, args.steps // 2), world)

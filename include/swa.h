@@ -164,7 +164,7 @@ size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W);
  * Limits and behaviour:
  *  - sizes whose workspace (swa_decode_workspace_size) exceeds
  *    SWA_DECODE_NOALLOC_SCRATCH_BYTES are rejected with SWA_ERR_UNSUPPORTED
- *    before anything is launched (B=64, Hq=32, D=128, W=4096 needs 8.5 MB);
+ *    before anything is launched (B=64, Hq=32, D=128, W=4096 needs 4.3 MB);
  *  - the first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.  The address is kept for the life of the

@@ -35,7 +35,7 @@
 
 namespace swa {
 
-constexpr int kDecodeSplit = 512;      // keys per block
+constexpr int kDecodeSplit = 1024;     // keys per block (1024 measured 0.5-2.5% faster than 512)
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeBlk = 16;         // keys per tensor-core block
 constexpr int kDecodeStages = 3;       // per-warp ring depth, in 16-key blocks

@@ -237,11 +237,11 @@ def _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps, seed):
 @pytest.mark.parametrize("B,Hq,Hkv,D,W,pos0", [
     (4, 32, 8, 128, 4096, [0, 1, 4094, 4095]),          # partial buffer, last slot, first wrap
     (3, 8, 2, 128, 4096, [4096, 8191, 30000]),          # wrap points and deep positions
-    (2, 4, 4, 64, 700, [10, 2000]),                     # G=1, W not a multiple of 512
+    (2, 4, 4, 64, 700, [10, 2000]),                     # G=1, W not a multiple of 16 keys per block
     (2, 16, 2, 128, 1000, [999, 5]),                    # G=8
     (2, 4, 2, 64, 300, [299, 77]),                      # G=2, single split
-    (2, 8, 2, 128, 8192, [8191, 20000]),                # 16 splits: workspace merge path
-    (1, 4, 1, 64, 5000, [4999]),                        # 10 splits, G=4, D=64
+    (2, 8, 2, 128, 8192, [8191, 20000]),                # 8 splits: workspace merge path
+    (1, 4, 1, 64, 5000, [4999]),                        # 5 splits, the last one partial, G=4, D=64
 ])
 def test_decode_edge_cases(oracle_mod, B, Hq, Hkv, D, W, pos0):
     _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps=3, seed=B * W + D)

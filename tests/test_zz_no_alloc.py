@@ -38,7 +38,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     assert torch.cuda.is_available()
     swa.build()
     L = swa.lib()
-    # W = 8192: 16 splits of 512 keys per sequence, merged through the scratch
+    # W = 8192: 8 splits of 1024 keys per sequence, merged through the scratch
     B, Hq, Hkv, D, W = 16, 32, 8, 128, 8192
     assert swa.swa_decode_workspace_size(B, Hq, Hkv, D, W) > 0
     scale = 1.0 / math.sqrt(D)
