@@ -197,10 +197,14 @@ swa_status_t swa_prefill_varlen(const void *q, const void *k, const void *v, voi
 
 /* swa_prefill_chunk_varlen -- one pre-fill chunk per sequence through its
  * rolling buffer (k_cache, v_cache [B, W, Hkv, D]), sequence b starting at
- * position start_pos[b].  A sequence of length 1 is a decode step (append,
- * then attend), so pre-fill chunks and decode tokens share one launch.  Any
- * length is accepted: a sequence longer than W leaves its last W positions in
- * the buffer.  Attend first, then write. */
+ * position start_pos[b].  A sequence of length 1 is a decode step (it sees
+ * its own key and the W-1 positions before it), so pre-fill chunks and decode
+ * tokens share one call.  Any length is accepted: a sequence longer than W
+ * leaves its last W positions in the buffer.  Attend first, then write.
+ * With group sizes Hq/Hkv of 1, 2, 4 or 8 the length-1 sequences are computed
+ * by the decode kernel (reading their own key and value from the packed k/v
+ * rows) and the others by the prefill kernel; with other group sizes the
+ * prefill kernel takes them all.  Up to three kernels on `stream`. */
 swa_status_t swa_prefill_chunk_varlen(const void *q, const void *k, const void *v, void *k_cache,
                                       void *v_cache, const int32_t *start_pos,
                                       const int32_t *cu_seqlens, void *out, int B, int total,

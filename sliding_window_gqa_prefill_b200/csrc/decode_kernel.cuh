@@ -107,36 +107,59 @@ __device__ __forceinline__ uint32_t swz_off(int r, int ch, int row_bytes) {
 // Partial result of one (sequence, kv head, split): per head m (base-2 max),
 // l (sum of 2^(s-m)) and o[D] (sum of 2^(s-m) v).  Layout in the workspace:
 // ml[((b*Hkv + g)*nsplit_max + s)*G + h] = {m, l};  o[...*D + d].
-// SINKS: keys past the window's come from the sink buffer (attention sinks);
-// compiled out of the plain decode.
-template <int D, int G, bool SINKS>
+// MODE 0: the window only.  MODE 1 (attention sinks): keys past the window's
+// come from the sink buffer.  MODE 2 (the length-1 sequences of a packed
+// chunk batch, attend before the buffer write): sequence b is decoded only if
+// it holds exactly one of the `total` packed rows (cu[b+1] - cu[b] == 1); its
+// q and out rows are row cu[b]; the buffer gives positions p-Lc .. p-1
+// (Lc = min(p, W-1), slot = position mod W) and the token's own key and value
+// are row cu[b] of the packed k and v, passed as ksink / vsink.  One block
+// covers the whole window, so no workspace is needed.
+constexpr int kDecodeWindow = 0, kDecodeSinks = 1, kDecodePackedRows = 2;
+
+template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
 swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kc,
                   const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ pos,
                   __nv_bfloat16 *__restrict__ out, float2 *__restrict__ ws_ml,
                   float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2,
                   int rope, const RopeTable rope_freq, const __nv_bfloat16 *__restrict__ ksink,
-                  const __nv_bfloat16 *__restrict__ vsink, int S) {
+                  const __nv_bfloat16 *__restrict__ vsink, int S, const int32_t *__restrict__ cu,
+                  int total) {
+    constexpr bool SINKS = MODE == kDecodeSinks;
     using Cfg = DecodeCfg<D, G>;
     constexpr int CH = Cfg::CH, RB = Cfg::ROW_BYTES;
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int Hq = Hkv * G;
+    int qrow = b;                                   // row of q and out
+    if (MODE == kDecodePackedRows) {
+        const int c0 = __ldg(cu + b), c1 = __ldg(cu + b + 1);
+        // not a single-row sequence (malformed offsets are recorded by the
+        // attention kernel that handles the other rows)
+        if (c1 - c0 != 1 || c0 < 0 || c1 > total) return;
+        qrow = c0;
+    }
     const int p = __ldg(pos + b);
     if (p < 0) {                                    // invalid position: record, write nothing
         if (threadIdx.x == 0 && split == 0 && g == 0) record_status(kStatusInvalid);
         return;
     }
-    const int Lw = (p >= W - 1) ? W : p + 1;           // keys in the rolling buffer
+    const int Lw = (p >= W - 1) ? W : p + 1;           // keys in the window
+    // MODE 2: keys 0 .. Lc-1 are buffer slots from that of position p - Lc
+    // on, key Lc the packed row
+    const int Lc = Lw - 1;
+    const int slot0 = (MODE == kDecodePackedRows) ? (int)((p - Lc) % W) : 0;
     // sink positions that left the window: slots 0 .. ns-1 of the sink buffer,
     // numbered after the window's keys
     const int ns = (SINKS && S > 0 && p >= W) ? min(S, p - W + 1) : 0;
     const int L = Lw + ns;
-    const int begin = split * kDecodeSplit;
+    const int split_keys = (MODE == kDecodePackedRows) ? L : kDecodeSplit;
+    const int begin = split * split_keys;
     if (begin >= L) return;
-    const int end = min(L, begin + kDecodeSplit);
-    const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
+    const int end = min(L, begin + split_keys);
+    const int nsplit = (L + split_keys - 1) / split_keys;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hr = lane >> 2;                // fragment row: head of the group (valid if < G)
@@ -148,13 +171,13 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     // with rope, each pair (2i, 2i+1) rotated at position p in fp32 first
     uint32_t qa[Cfg::KSTEPS][2];
     {
-        const __nv_bfloat16 *qrow = q + ((size_t)b * Hq + g * G + (head_ok ? hr : 0)) * D;
+        const __nv_bfloat16 *qp = q + ((size_t)qrow * Hq + g * G + (head_ok ? hr : 0)) * D;
 #pragma unroll
         for (int kk = 0; kk < Cfg::KSTEPS; ++kk)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int d = kk * 16 + hf * 8 + 2 * t4;
-                uint32_t w = head_ok ? __ldg(reinterpret_cast<const uint32_t *>(qrow + d)) : 0u;
+                uint32_t w = head_ok ? __ldg(reinterpret_cast<const uint32_t *>(qp + d)) : 0u;
                 if (rope && head_ok) {
                     float c, sn;
                     rope_cos_sin((double)p, rope_freq.f[d >> 1], c, sn);
@@ -170,6 +193,8 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv + g) * D;
     const __nv_bfloat16 *ksbase = ns ? ksink + ((size_t)b * S * Hkv + g) * D : kbase;
     const __nv_bfloat16 *vsbase = ns ? vsink + ((size_t)b * S * Hkv + g) * D : vbase;
+    const __nv_bfloat16 *knew = (MODE == kDecodePackedRows) ? ksink + ((size_t)qrow * Hkv + g) * D : kbase;
+    const __nv_bfloat16 *vnew = (MODE == kDecodePackedRows) ? vsink + ((size_t)qrow * Hkv + g) * D : vbase;
 
     const int nblk = (end - begin + kDecodeBlk - 1) / kDecodeBlk;
     const int my_blocks = (nblk > warp) ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
@@ -189,6 +214,18 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                 const size_t rowi = (size_t)(key - Lw) * row_stride + ch * 8;
                 cp_async16(st + off, ksbase + rowi);
                 cp_async16(st + Cfg::BLK_BYTES + off, vsbase + rowi);
+            } else if (MODE == kDecodePackedRows) {
+                if (key == Lc) {
+                    cp_async16(st + off, knew + ch * 8);
+                    cp_async16(st + Cfg::BLK_BYTES + off, vnew + ch * 8);
+                } else {
+                    const long long sl = (long long)slot0 + key;
+                    const int slot = (int)(sl >= W ? sl - W : sl);
+                    if (!in_bounds(slot, W)) continue;
+                    const size_t rowi = (size_t)slot * row_stride + ch * 8;
+                    cp_async16(st + off, kbase + rowi);
+                    cp_async16(st + Cfg::BLK_BYTES + off, vbase + rowi);
+                }
             } else {
                 if (!in_bounds(key, W)) continue;
                 const size_t rowi = (size_t)key * row_stride + ch * 8;
@@ -319,8 +356,9 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             acc += src[d] * sc;
         }
         if (nsplit == 1) {
-            const size_t oi = ((size_t)b * Hq + g * G + h) * D + d;
-            if (in_bounds((long long)oi, (long long)gridDim.z * Hq * D)) out[oi] = __float2bfloat16_rn(acc / l);
+            const size_t oi = ((size_t)qrow * Hq + g * G + h) * D + d;
+            const long long rows = (MODE == kDecodePackedRows) ? total : gridDim.z;
+            if (in_bounds((long long)oi, rows * Hq * D)) out[oi] = __float2bfloat16_rn(acc / l);
         } else {
             const size_t slot = ((size_t)(b * Hkv + g) * nsplit_max + split) * G + h;
             if (!in_bounds(split, nsplit_max)) continue;

@@ -64,6 +64,9 @@ struct PrefillParams {
     // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
     // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
     const int32_t *cu_seqlens;
+    // variable-length chunk batch: 1 leaves sequences of one row to the
+    // decode kernel (no work units for them)
+    int skip_len1;
     // attention sinks (one-shot prefill): positions j < sinks stay visible to
     // every query besides its window
     int sinks;
@@ -365,12 +368,14 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init_fence();
         if (p.cu_seqlens) {
             // query blocks per sequence, prefix-summed (empty or malformed
-            // sequences count as empty; malformed ones are recorded)
+            // sequences count as empty; malformed ones are recorded; with
+            // skip_len1, sequences of one row too)
             int acc = 0;
             for (int b = 0; b < p.B; ++b) {
                 pre[b] = acc;
-                const int n = varlen_rows(p, b);
+                int n = varlen_rows(p, b);
                 if (n == 0 && __ldg(p.cu_seqlens + b + 1) != __ldg(p.cu_seqlens + b)) record_status(kStatusInvalid);
+                if (n == 1 && p.skip_len1) n = 0;
                 acc += (n + 127) / 128;
             }
             pre[p.B] = acc;

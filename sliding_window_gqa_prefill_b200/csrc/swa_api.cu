@@ -97,10 +97,13 @@ swa_status_t device_info(DeviceInfo **out) {
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           swa::PrefillCfg<128>::SMEM_ALLOC));
 #define SWA_SET_DECODE_ATTR(DD, GG)                                                           \
-    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, false>,                 \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, swa::kDecodeWindow>,    \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,           \
                                       swa::DecodeCfg<DD, GG>::SMEM_BYTES));                  \
-    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, true>,                  \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, swa::kDecodeSinks>,     \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                      swa::DecodeCfg<DD, GG>::SMEM_BYTES));                  \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, swa::kDecodePackedRows>, \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,           \
                                       swa::DecodeCfg<DD, GG>::SMEM_BYTES));
         SWA_SET_DECODE_ATTR(64, 1) SWA_SET_DECODE_ATTR(64, 2) SWA_SET_DECODE_ATTR(64, 4)
@@ -182,12 +185,14 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
     float2 *ws_ml = ws ? reinterpret_cast<float2 *>(static_cast<char *>(ws) + ((o_elems * 4 + 255) & ~size_t(255)))
                        : nullptr;
     dim3 grid(nsm, Hkv, B);
-    auto kernel = S > 0 ? swa::swa_decode_kernel<D, G, true> : swa::swa_decode_kernel<D, G, false>;
+    auto kernel = S > 0 ? swa::swa_decode_kernel<D, G, swa::kDecodeSinks>
+                        : swa::swa_decode_kernel<D, G, swa::kDecodeWindow>;
     kernel<<<grid, swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
         static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
         Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{},
-        static_cast<const __nv_bfloat16 *>(ksink), static_cast<const __nv_bfloat16 *>(vsink), S);
+        static_cast<const __nv_bfloat16 *>(ksink), static_cast<const __nv_bfloat16 *>(vsink), S,
+        nullptr, 0);
     SWA_CUDA_TRY(cudaGetLastError());
     if (nsm > 1) {
         swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), G * D, 0, s>>>(
@@ -208,6 +213,37 @@ swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *v
         case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         default: return SWA_ERR_UNSUPPORTED;
+    }
+}
+
+// The length-1 sequences of a packed chunk batch (q/k/v/out [total, H, D]),
+// one block per (sequence, kv head); the other sequences' blocks return at once.
+template <int D, int G>
+swa_status_t launch_decode_packed_dg(const void *q, const void *k, const void *v, const void *kc,
+                                     const void *vc, const int32_t *start_pos, const int32_t *cu,
+                                     void *out, int B, int total, int Hkv, int W, float scale,
+                                     cudaStream_t s) {
+    swa::swa_decode_kernel<D, G, swa::kDecodePackedRows>
+        <<<dim3(1, Hkv, B), swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
+            static_cast<const __nv_bfloat16 *>(vc), start_pos, static_cast<__nv_bfloat16 *>(out), nullptr,
+            nullptr, Hkv, W, 1, scale * kLog2e, 0, swa::RopeTable{}, static_cast<const __nv_bfloat16 *>(k),
+            static_cast<const __nv_bfloat16 *>(v), 0, cu, total);
+    SWA_CUDA_TRY(cudaGetLastError());
+    return SWA_OK;
+}
+
+// false when the decode kernel has no instance for this head group
+template <int D>
+bool launch_decode_packed_d(int G, swa_status_t *e, const void *q, const void *k, const void *v,
+                            const void *kc, const void *vc, const int32_t *start_pos, const int32_t *cu,
+                            void *out, int B, int total, int Hkv, int W, float scale, cudaStream_t s) {
+    switch (G) {
+        case 1: *e = launch_decode_packed_dg<D, 1>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 2: *e = launch_decode_packed_dg<D, 2>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 4: *e = launch_decode_packed_dg<D, 4>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 8: *e = launch_decode_packed_dg<D, 8>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        default: return false;
     }
 }
 
@@ -388,6 +424,17 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
         if (swa_status_t e = make_operand_map(&mvs, v_sink, D, Hkv, S, B)) return e;
     }
     p.sink_buf = S;
+    if (cu_seqlens) {
+        // length-1 sequences (decode tokens) go to the decode kernel, which
+        // reads their windows at memory speed instead of as 128-row tiles
+        swa_status_t ed = SWA_OK;
+        const bool dec = D == 128 ? launch_decode_packed_d<128>(G, &ed, q, k, v, k_cache, v_cache, start_pos,
+                                                                cu_seqlens, out, B, C, Hkv, W, scale, s)
+                                  : launch_decode_packed_d<64>(G, &ed, q, k, v, k_cache, v_cache, start_pos,
+                                                               cu_seqlens, out, B, C, Hkv, W, scale, s);
+        if (ed) return ed;
+        p.skip_len1 = dec ? 1 : 0;
+    }
     swa_status_t e = D == 128 ? launch_prefill<128>(mq, mk, mv, mkc, mvc, mks, mvs, p, dev->sms, s)
                               : launch_prefill<64>(mq, mk, mv, mkc, mvc, mks, mvs, p, dev->sms, s);
     if (e) return e;

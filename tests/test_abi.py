@@ -88,8 +88,9 @@ def test_null_and_bad_sizes_rejected_without_device(lib):
 def test_workspace_size_and_status_strings(lib):
     assert lib.swa_decode_workspace_size(0, 32, 8, 128, 4096) == 0
     n = lib.swa_decode_workspace_size(64, 32, 8, 128, 4096)
-    # (B*Hq*splits) rows of D floats, then one (m, l) pair per row
-    rows = 64 * 32 * 8
+    # (B*Hq*splits) rows of D floats, then one (m, l) pair per row; the
+    # 4096-key window takes 4 splits of 1024 keys
+    rows = 64 * 32 * 4
     assert n == ((rows * 128 * 4 + 255) // 256) * 256 + rows * 8
     assert lib.swa_status_string(0) == b"SWA_OK"
     assert lib.swa_status_string(4) == b"SWA_ERR_TIMEOUT"

@@ -1,7 +1,9 @@
 """Variable-length batches in one launch against the fp64 oracle run per
-sequence: packed one-shot prefill, and a mixed call in which some sequences
+sequence: packed one-shot prefill, and mixed calls in which some sequences
 pre-fill a chunk (through their rolling buffer), some decode one token, one
-chunk is longer than the window and one sequence is empty."""
+chunk is longer than the window and one sequence is empty.  The one-token
+sequences go to the decode kernel for group sizes 1, 2, 4 and 8 and stay in
+the attention kernel for the others (3 and 6 here); both are checked."""
 import math
 
 import numpy as np
@@ -55,36 +57,32 @@ def test_prefill_varlen_matches_per_sequence_oracle(oracle_mod, lens, Hq, Hkv, D
         close(out[s:e], ref[0], f"varlen seq {b} (n={n})")
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (6, 2), (6, 1)])   # group sizes 4, 3 and 6
-def test_mixed_chunks_and_decode_in_one_launch(oracle_mod, Hq, Hkv):
-    D, W = 128, 256
+def _mixed(oracle_mod, hist, now, Hq, Hkv, D, W, seed):
+    """One swa_prefill_chunk_varlen call: sequence b has hist[b] positions in
+    its buffer (written through the oracle's write rule) and now[b] tokens in
+    the call; every output row against the oracle's chunk attention, then the
+    buffers bit for bit against the oracle's write."""
     scale = 1 / math.sqrt(D)
-    # per sequence: history length already in the buffer, tokens in this call
-    hist = [1000, 7000, 0, 300, 50]
-    now = [500, 1, 300, 0, 1]
     B = len(hist)
-    rng_seed = 90
-    kc = torch.zeros(B, W, Hkv, D, dtype=torch.bfloat16)
-    vc = torch.zeros_like(kc)
-    kref, vref = f64(kc), f64(vc)
+    kref = np.zeros((B, W, Hkv, D))
+    vref = np.zeros_like(kref)
     sp = np.full((B, W), -1, np.int32)
-    # fill each buffer with its history through the oracle's write rule
     for b in range(B):
-        if hist[b] == 0:
+        n = min(hist[b], W)                  # older positions would be overwritten
+        if n == 0:
             continue
-        kh = wl.random_bf16((1, hist[b], Hkv, D), rng_seed + b)
-        vh = wl.random_bf16((1, hist[b], Hkv, D), rng_seed + 50 + b)
+        kh = wl.random_bf16((1, n, Hkv, D), seed + b)
+        vh = wl.random_bf16((1, n, Hkv, D), seed + 500 + b)
         kb, vb, spb = kref[b:b + 1].copy(), vref[b:b + 1].copy(), sp[b:b + 1].copy()
-        oracle_mod.cache_append(kb, vb, spb, f64(kh), f64(vh), [0])
+        oracle_mod.cache_append(kb, vb, spb, f64(kh), f64(vh), [hist[b] - n])
         kref[b], vref[b], sp[b] = kb[0], vb[0], spb[0]
-    kc = torch.from_numpy(kref).to(torch.bfloat16)
-    vc = torch.from_numpy(vref).to(torch.bfloat16)
+    kg = torch.from_numpy(kref).to(torch.bfloat16).cuda()
+    vg = torch.from_numpy(vref).to(torch.bfloat16).cuda()
     total = sum(now)
     cu = np.array([0] + list(np.cumsum(now)), np.int32)
-    q = wl.random_bf16((total, Hq, D), 95)
-    k = wl.random_bf16((total, Hkv, D), 96)
-    v = wl.random_bf16((total, Hkv, D), 97)
-    kg, vg = kc.cuda(), vc.cuda()
+    q = wl.random_bf16((total, Hq, D), seed + 1001)
+    k = wl.random_bf16((total, Hkv, D), seed + 1002)
+    v = wl.random_bf16((total, Hkv, D), seed + 1003)
     start = torch.tensor(hist, dtype=torch.int32)
     out = swa.swa_prefill_chunk_varlen(q.cuda(), k.cuda(), v.cuda(), kg, vg, start.cuda(),
                                        torch.from_numpy(cu).cuda(), W, scale)
@@ -101,3 +99,24 @@ def test_mixed_chunks_and_decode_in_one_launch(oracle_mod, Hq, Hkv):
         oracle_mod.cache_append(kb, vb, sp[b:b + 1].copy(), f64(k[s:e])[None], f64(v[s:e])[None], [hist[b]])
         kref[b], vref[b] = kb[0], vb[0]
     assert np.array_equal(f64(kg.cpu()), kref) and np.array_equal(f64(vg.cpu()), vref)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (6, 2), (6, 1)])   # group sizes 4, 3 and 6
+def test_mixed_chunks_and_decode_in_one_launch(oracle_mod, Hq, Hkv):
+    # per sequence: history length already in the buffer, tokens in this call
+    _mixed(oracle_mod, [1000, 7000, 0, 300, 50], [500, 1, 300, 0, 1], Hq, Hkv, 128, 256, 90)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_tokens_of_a_packed_batch(oracle_mod, G, D):
+    """Length-1 sequences of a chunk batch at positions around the buffer
+    edges (first token, just below the window, the wrap, far past it): with
+    group sizes 1, 2, 4 and 8 they are decoded by the decode kernel, which
+    takes the token's own key and value from the packed rows (its slot still
+    holds position p - W, or nothing, until the write after the attention);
+    two chunks and an empty sequence share the launch."""
+    W = 300
+    hist = [0, 1, W - 2, W - 1, W, W + 1, 2 * W - 1, 5000, 700, 0, 37]
+    now = [1, 1, 1, 1, 1, 1, 1, 1, 130, 0, 200]
+    _mixed(oracle_mod, hist, now, 2 * G, 2, D, W, 300 + 10 * G + D)
