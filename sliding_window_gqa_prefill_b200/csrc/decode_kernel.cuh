@@ -39,6 +39,10 @@ constexpr int kDecodeSplit = 1024;     // keys per block (1024 measured 0.5-2.5%
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeBlk = 16;         // keys per tensor-core block
 constexpr int kDecodeStages = 3;       // per-warp ring depth, in 16-key blocks
+// MODE 2 (length-1 sequences of a packed chunk batch, no workspace): the
+// window of one (sequence, kv head) is split over a cluster of this many
+// blocks, merged through distributed shared memory
+constexpr int kDecodeClusterSplits = 4;
 
 template <int D, int G>
 struct DecodeCfg {
@@ -51,8 +55,10 @@ struct DecodeCfg {
     static constexpr int CPL = kDecodeBlk * CH / 32;           // 16-byte copies per lane, K or V
     static constexpr int KSTEPS = D / 16;                      // MMA k-steps of S = Q K^T
     static constexpr int NB = D / 8;                           // 8-column blocks of O
-    // the warp merge reuses the rings once every copy has landed
-    static constexpr int MERGE_BYTES = kDecodeWarps * G * (D + 2) * 4;
+    // the warp merge reuses the rings once every copy has landed: per warp
+    // and head {o[D], m, l}, then the block's merged {o[D], m, l} per head
+    // (read by the cluster merge)
+    static constexpr int MERGE_BYTES = (kDecodeWarps + 1) * G * (D + 2) * 4;
     static constexpr int SMEM_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "group size 1, 2, 4 or 8");
@@ -113,8 +119,10 @@ __device__ __forceinline__ uint32_t swz_off(int r, int ch, int row_bytes) {
 // it holds exactly one of the `total` packed rows (cu[b+1] - cu[b] == 1); its
 // q and out rows are row cu[b]; the buffer gives positions p-Lc .. p-1
 // (Lc = min(p, W-1), slot = position mod W) and the token's own key and value
-// are row cu[b] of the packed k and v, passed as ksink / vsink.  One block
-// covers the whole window, so no workspace is needed.
+// are row cu[b] of the packed k and v, passed as ksink / vsink.  The window
+// is split over a cluster of kDecodeClusterSplits blocks (grid x), merged
+// through distributed shared memory (each block merges a quarter of the
+// outputs from all blocks' partials), so no workspace is needed.
 constexpr int kDecodeWindow = 0, kDecodeSinks = 1, kDecodePackedRows = 2;
 
 template <int D, int G, int MODE>
@@ -155,9 +163,12 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     // numbered after the window's keys
     const int ns = (SINKS && S > 0 && p >= W) ? min(S, p - W + 1) : 0;
     const int L = Lw + ns;
-    const int split_keys = (MODE == kDecodePackedRows) ? L : kDecodeSplit;
-    const int begin = split * split_keys;
-    if (begin >= L) return;
+    constexpr int kClusterKeys = kDecodeClusterSplits * kDecodeBlk;
+    const int split_keys =
+        (MODE == kDecodePackedRows) ? (L + kClusterKeys - 1) / kClusterKeys * kDecodeBlk : kDecodeSplit;
+    // MODE 2: a block past the window's keys still takes part in the merge
+    if (MODE != kDecodePackedRows && split * split_keys >= L) return;
+    const int begin = min(split * split_keys, L);
     const int end = min(L, begin + split_keys);
     const int nsplit = (L + split_keys - 1) / split_keys;
 
@@ -342,6 +353,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         }
     }
     __syncthreads();
+    float *part = mg + kDecodeWarps * G * (D + 2);  // [G][D+2]: the block's merge (MODE 2)
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D, d = idx % D;
         float m = -INFINITY;
@@ -355,16 +367,54 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             l += src[D + 1] * sc;
             acc += src[d] * sc;
         }
-        if (nsplit == 1) {
+        if (MODE == kDecodePackedRows) {
+            part[h * (D + 2) + d] = acc;
+            if (d == 0) {
+                part[h * (D + 2) + D] = m;
+                part[h * (D + 2) + D + 1] = l;
+            }
+        } else if (nsplit == 1) {
             const size_t oi = ((size_t)qrow * Hq + g * G + h) * D + d;
-            const long long rows = (MODE == kDecodePackedRows) ? total : gridDim.z;
-            if (in_bounds((long long)oi, rows * Hq * D)) out[oi] = __float2bfloat16_rn(acc / l);
+            if (in_bounds((long long)oi, (long long)gridDim.z * Hq * D)) out[oi] = __float2bfloat16_rn(acc / l);
         } else {
             const size_t slot = ((size_t)(b * Hkv + g) * nsplit_max + split) * G + h;
             if (!in_bounds(split, nsplit_max)) continue;
             ws_o[slot * D + d] = acc;
             if (d == 0) ws_ml[slot] = make_float2(m, l);
         }
+    }
+    if constexpr (MODE == kDecodePackedRows) {
+        // every block of the cluster reaches both barriers: the only returns
+        // above depend on (b) alone, which the cluster shares
+        cluster_sync_all();
+        {   // each block of the cluster merges and writes a quarter of the outputs
+            static_assert((G * D) % kDecodeClusterSplits == 0, "outputs per block");
+            constexpr int kPer = G * D / kDecodeClusterSplits;
+            const int i0 = (int)cluster_rank() * kPer;
+            for (int idx = i0 + threadIdx.x; idx < i0 + kPer; idx += blockDim.x) {
+                const int h = idx / D, d = idx % D;
+                const uint32_t row = smem_addr(part + h * (D + 2));
+                float mr[kDecodeClusterSplits], lr[kDecodeClusterSplits], ar[kDecodeClusterSplits];
+                float m = -INFINITY;
+#pragma unroll
+                for (int r = 0; r < kDecodeClusterSplits; ++r) {
+                    mr[r] = ld_peer_f32(row + D * 4, r);
+                    lr[r] = ld_peer_f32(row + (D + 1) * 4, r);
+                    ar[r] = ld_peer_f32(row + d * 4, r);
+                    m = fmaxf(m, mr[r]);
+                }
+                float l = 0.f, acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < kDecodeClusterSplits; ++r) {
+                    const float sc = (mr[r] == -INFINITY) ? 0.f : ex2_approx(mr[r] - m);
+                    l += lr[r] * sc;
+                    acc += ar[r] * sc;
+                }
+                const size_t oi = ((size_t)qrow * Hq + g * G + h) * D + d;
+                if (in_bounds((long long)oi, (long long)total * Hq * D)) out[oi] = __float2bfloat16_rn(acc / l);
+            }
+        }
+        cluster_sync_all();                          // peers' shared memory stays until read
     }
 }
 

@@ -142,6 +142,35 @@ __device__ __forceinline__ bool mbar_drain_bounded(uint32_t bar, uint32_t parity
 }
 
 // ---------------------------------------------------------------------------
+// Thread-block clusters: rank, a barrier of all threads of all blocks, and
+// loads from a peer block's shared memory (distributed shared memory).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Release / acquire: shared-memory writes before it are visible to every
+// block of the cluster after it.  Every thread of every block must reach it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address, in the cluster window, of the same shared-memory offset in block `rank`.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local_addr, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+    return a;
+}
+
+__device__ __forceinline__ float ld_peer_f32(uint32_t local_addr, uint32_t rank) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(peer_addr(local_addr, rank)) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------------------
 // TMA: tiled 4-D tensor load into shared memory, completion on an mbarrier.
 // Coordinates are element indices, innermost first.  No multicast.
 // ---------------------------------------------------------------------------

@@ -216,20 +216,37 @@ swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *v
     }
 }
 
-// The length-1 sequences of a packed chunk batch (q/k/v/out [total, H, D]),
-// one block per (sequence, kv head); the other sequences' blocks return at once.
+// The length-1 sequences of a packed chunk batch (q/k/v/out [total, H, D]):
+// a cluster of kDecodeClusterSplits blocks per (sequence, kv head), merged in
+// distributed shared memory; the other sequences' blocks return at once.
 template <int D, int G>
 swa_status_t launch_decode_packed_dg(const void *q, const void *k, const void *v, const void *kc,
                                      const void *vc, const int32_t *start_pos, const int32_t *cu,
                                      void *out, int B, int total, int Hkv, int W, float scale,
                                      cudaStream_t s) {
-    swa::swa_decode_kernel<D, G, swa::kDecodePackedRows>
-        <<<dim3(1, Hkv, B), swa::kDecodeWarps * 32, swa::DecodeCfg<D, G>::SMEM_BYTES, s>>>(
-            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
-            static_cast<const __nv_bfloat16 *>(vc), start_pos, static_cast<__nv_bfloat16 *>(out), nullptr,
-            nullptr, Hkv, W, 1, scale * kLog2e, 0, swa::RopeTable{}, static_cast<const __nv_bfloat16 *>(k),
-            static_cast<const __nv_bfloat16 *>(v), 0, cu, total);
-    SWA_CUDA_TRY(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(swa::kDecodeClusterSplits, Hkv, B);
+    cfg.blockDim = dim3(swa::kDecodeWarps * 32);
+    cfg.dynamicSmemBytes = swa::DecodeCfg<D, G>::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = swa::kDecodeClusterSplits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q);
+    const __nv_bfloat16 *kcb = static_cast<const __nv_bfloat16 *>(kc);
+    const __nv_bfloat16 *vcb = static_cast<const __nv_bfloat16 *>(vc);
+    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(k);
+    const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(v);
+    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(out);
+    float2 *no_ml = nullptr;
+    float *no_o = nullptr;
+    SWA_CUDA_TRY(cudaLaunchKernelEx(&cfg, swa::swa_decode_kernel<D, G, swa::kDecodePackedRows>, qb, kcb, vcb,
+                                    start_pos, ob, no_ml, no_o, Hkv, W, 1, scale * kLog2e, 0, swa::RopeTable{},
+                                    kb, vb, 0, cu, total));
     return SWA_OK;
 }
 

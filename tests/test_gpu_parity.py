@@ -198,6 +198,7 @@ def _chunked_case(oracle_mod, B, N, C, Hq, Hkv, D, W, seed, start=0):
     (1, 333, 45, 2, 1, 128, 100),     # small ragged chunks
     (1, 1100, 300, 6, 2, 128, 384),   # odd group, wrap inside tiles
     (2, 2560, 1280, 16, 4, 128, 1536),  # 160 units: on 148 SMs the last 12 run as single-head units
+    (1, 2560, 1280, 32, 16, 64, 1280),  # the same split with G=2, D=64, C=W
 ])
 def test_chunked_prefill_matches_oracle(oracle_mod, B, N, C, Hq, Hkv, D, W):
     q, k, v, scale, out, kc, vc = _chunked_case(oracle_mod, B, N, C, Hq, Hkv, D, W, seed=N + C)

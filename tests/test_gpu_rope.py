@@ -91,11 +91,14 @@ def test_prefill_rope_fused_q(oracle_mod, B, N, Hq, Hkv, D, W):
     close(out, ref, "prefill rope")
 
 
-def test_chunked_rope_then_decode_rope_continue_the_sequence(oracle_mod):
+@pytest.mark.parametrize("B,N,C,Hq,Hkv,D,W", [
+    (2, 520, 200, 8, 2, 128, 256),
+    (1, 2560, 1280, 32, 4, 64, 1280),    # 160 units: the last wave split into single-head units, G=8, D=64
+])
+def test_chunked_rope_then_decode_rope_continue_the_sequence(oracle_mod, B, N, C, Hq, Hkv, D, W):
     """Chunks with q rotated at load and keys rotated before the chunk call,
     then decode with the key rotated into the cache and q rotated in the
     kernel: every output equals one-shot SWA on exactly rotated q and k."""
-    B, N, C, Hq, Hkv, D, W = 2, 520, 200, 8, 2, 128, 256
     q = wl.random_bf16((B, N + 2, Hq, D), 69)
     k = wl.random_bf16((B, N + 2, Hkv, D), 70)
     v = wl.random_bf16((B, N + 2, Hkv, D), 71)

@@ -85,6 +85,7 @@ def test_streaming_decode_with_sinks(oracle_mod, W, S, D):
     (1, 900, 256, 8, 2, 128, 256, 4),     # C = W
     (2, 700, 100, 4, 4, 64, 128, 8),      # C < W, MHA, D=64
     (1, 1000, 300, 6, 2, 128, 384, 130),  # two sink tiles, odd group
+    (2, 2560, 1280, 16, 4, 128, 1536, 4),  # last wave split into single-head units, with a sink tile
 ])
 def test_chunked_prefill_with_sinks(oracle_mod, B, N, C, Hq, Hkv, D, W, S):
     """Chunks through the rolling buffer with the sink buffer: the outputs equal
