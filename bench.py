@@ -613,9 +613,20 @@ def measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, iters, world):
         swa.swa_cache_append_sinks(kn, vn, kc, vc, ks, vs, pos)
         swa.swa_decode_sinks(qd, kc, vc, ks, vs, pos, dw.scale, out=od, workspace=ws)
 
+    # timed as the decode of the step runs: 16 steps (the same position each
+    # time) captured in one CUDA graph and replayed
+    reps = 16
     for name, fn in (("decode_rope_step", dec_rope), ("decode_sinks4_step", dec_sinks)):
-        ms = max_over_ranks(_time_ms(fn, iters * 4), world)
-        res[name] = {"tokens_per_s": dw.B * world / (ms * 1e-3), "us": ms * 1e3}
+        fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(reps):
+                fn()
+        ms = max_over_ranks(_time_ms(graph.replay, iters), world) / reps
+        del graph
+        res[name] = {"tokens_per_s": dw.B * world / (ms * 1e-3), "us": ms * 1e3,
+                     "note": "append + decode (+ split merge) per step, replayed from a 16-step CUDA graph"}
     # mixed launch: 4 sequences pre-fill a 4096-token chunk, 60 decode one token
     nseq, nchunk, C = 64, 4, 4096
     lens = [C] * nchunk + [1] * (nseq - nchunk)

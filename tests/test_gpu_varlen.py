@@ -120,3 +120,34 @@ def test_decode_tokens_of_a_packed_batch(oracle_mod, G, D):
     hist = [0, 1, W - 2, W - 1, W, W + 1, 2 * W - 1, 5000, 700, 0, 37]
     now = [1, 1, 1, 1, 1, 1, 1, 1, 130, 0, 200]
     _mixed(oracle_mod, hist, now, 2 * G, 2, D, W, 300 + 10 * G + D)
+
+
+def test_mixed_call_replays_from_a_cuda_graph():
+    """A serving loop captures the mixed call (decode clusters, attention
+    kernel, buffer write) in a CUDA graph: one replay gives the eager call's
+    outputs and buffers bit for bit."""
+    Hq, Hkv, D, W = 8, 2, 128, 256
+    hist = [0, 300, 9000, 40, 700]
+    now = [130, 1, 1, 1, 200]
+    B, total = len(hist), sum(now)
+    cu = torch.tensor([0] + list(np.cumsum(now)), dtype=torch.int32).cuda()
+    start = torch.tensor(hist, dtype=torch.int32).cuda()
+    q = wl.random_bf16((total, Hq, D), 501).cuda()
+    k = wl.random_bf16((total, Hkv, D), 502).cuda()
+    v = wl.random_bf16((total, Hkv, D), 503).cuda()
+    kc0 = wl.random_bf16((B, W, Hkv, D), 504).cuda()
+    vc0 = wl.random_bf16((B, W, Hkv, D), 505).cuda()
+    kc, vc = kc0.clone(), vc0.clone()
+    ref = swa.swa_prefill_chunk_varlen(q, k, v, kc, vc, start, cu, W, 0.09)
+    torch.cuda.synchronize()
+    kg, vg = kc0.clone(), vc0.clone()
+    out = torch.empty_like(q)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        swa.swa_prefill_chunk_varlen(q, k, v, kg, vg, start, cu, W, 0.09, out=out)
+    kg.copy_(kc0)
+    vg.copy_(vc0)
+    graph.replay()
+    torch.cuda.synchronize()
+    del graph
+    assert torch.equal(out, ref) and torch.equal(kg, kc) and torch.equal(vg, vc)
