@@ -45,6 +45,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
+    ap.add_argument("--log", default=None,
+                    help="also append the result, and one row per measured part, as JSON lines to this file")
     ap.add_argument("--ncu-case", choices=["prefill", "prefill_b2", "chunk", "decode"], default=None,
                     help="run a reduced case of one kernel three times for an ncu capture (no timing)")
     return ap.parse_args(argv)
@@ -188,9 +190,11 @@ def barrier(world: int):
 
 def bench_config(hp, world: int) -> dict:
     """The workload description both arms print (native and reference)."""
+    from sliding_window_gqa_prefill_b200 import workloads as wl
     return {
         "workload": hp.name,
         "B": hp.B, "N": hp.N, "W": hp.W, "Hq": hp.Hq, "Hkv": hp.Hkv, "D": hp.D,
+        "seeds": {"prefill": hp.seed, "chunked": wl.CHUNKED_16K.seed, "decode": wl.DECODE_B64.seed},
         "parallelism": f"replicas{world}" if world > 1 else "single",
         "l2": "inputs larger than L2 (prefill q/k/v/out 640 MB, decode cache 1 GB); no flush",
         "step": "one-shot prefill + 4-chunk prefill (N=16384) + 128 decode steps (B=64, graph)",
@@ -208,10 +212,12 @@ NOMINAL_BF16_TFLOPS = 2250.0
 _ORACLE_CACHE = {}
 
 
-def cpu_oracle_sample(target_s: float):
+def cpu_oracle_sample(target_s: float, gpu_out=None):
     """Time the fp64 oracle on a row sample of the headline prefill workload.
 
-    Returns (TFLOP/s, seconds, rows, threads)."""
+    Returns (TFLOP/s, seconds, rows, threads, check): with gpu_out (the GPU's
+    output of the same seeded workload, [B, N, Hq, D]) check holds the error
+    of the GPU's rows against the oracle's on the sampled rows, else None."""
     import numpy as np
     import oracle
     from sliding_window_gqa_prefill_b200 import workloads as wl
@@ -226,11 +232,18 @@ def cpu_oracle_sample(target_s: float):
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     done, t_total, used = 0, 0.0, 0
     batch = 8
+    err_max, err_sum, err_n = 0.0, 0.0, 0
     while t_total < target_s and used + batch <= pool.size:
         rows = pool[used:used + batch]
         t0 = time.perf_counter()
-        oracle.swa_prefill(qn, kn, vn, w.W, w.scale, rows=rows)
+        ref = oracle.swa_prefill(qn, kn, vn, w.W, w.scale, rows=rows)
         dt = time.perf_counter() - t0
+        if gpu_out is not None:            # outside the timed region
+            got = gpu_out[:, rows.tolist()].float().cpu().numpy().astype(np.float64)
+            err = np.abs(got - ref)
+            err_max = max(err_max, float(err.max()))
+            err_sum += float(err.sum())
+            err_n += err.size
         t_total += dt
         used += batch
         done += batch
@@ -240,7 +253,11 @@ def cpu_oracle_sample(target_s: float):
             if batch <= 0:
                 break
     flops = 4.0 * w.B * w.Hq * w.D * w.W * done
-    return flops / t_total / 1e12, t_total, done, threads
+    check = None
+    if gpu_out is not None and err_n:
+        check = {"rows": done, "max_abs": err_max, "mean_abs": err_sum / err_n, "bar": [2e-2, 2e-3],
+                 "within_bar": err_max <= 2e-2 and err_sum / err_n <= 2e-3}
+    return flops / t_total / 1e12, t_total, done, threads, check
 
 
 # ---------------------------------------------------------------- native GPU run
@@ -434,10 +451,12 @@ def run_native(args):
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            tf, secs, rows, thr = cpu_oracle_sample(args.cpu_seconds)
+            tf, secs, rows, thr, check = cpu_oracle_sample(args.cpu_seconds, gpu_out=out)
             cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                    "sample": f"{rows} query rows x B={hp.B} x {hp.Hq} heads of the headline prefill "
                              f"(each row W={hp.W} keys), fp64, {secs:.1f} s"}
+            if check is not None:       # the timed step's own output on the sampled rows
+                cpu["check_of_timed_output"] = check
         traffic = ncu_traffic("swa_prefill_kernel<128>")
         result = {
             "metric": METRIC,
@@ -658,10 +677,10 @@ def run_reference(args):
     hp = wl.HEADLINE_PREFILL
     per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_sample(per_step / 4)
+        cpu_oracle_sample(per_step / 4)  # warm-up
     vals, secs, rows_total, thr = [], 0.0, 0, 1
     for _ in range(args.steps):
-        tf, s, rows, thr = cpu_oracle_sample(per_step)
+        tf, s, rows, thr, _ = cpu_oracle_sample(per_step)
         vals.append(tf)
         secs += s
         rows_total += rows
@@ -760,6 +779,25 @@ def main(argv=None):
         res = run_native(args)
     if res is not None:
         print(json.dumps(res), flush=True)
+        if args.log:
+            write_log(args.log, res)
+
+
+def write_log(path: str, res: dict) -> None:
+    """Append the result line, then one row per measured part (each with the
+    workload config, so that rows stand alone), as JSON lines."""
+    rows = [res]
+    base = {"impl": res.get("impl", "native"), "config": res.get("config"), "clocks": res.get("clocks")}
+    for part in ("decode", "chunked", "roofline", "roofline_prefill", "e2e", "cpu_baseline"):
+        if isinstance(res.get(part), dict):
+            rows.append({"part": part, **base, **res[part]})
+    for group in ("extras", "sweep"):
+        for name, val in (res.get(group) or {}).items():
+            rows.append({"part": f"{group}.{name}", **base,
+                         **(val if isinstance(val, dict) else {"value": val})})
+    with open(path, "a") as f:
+        for r in rows:
+            f.write(json.dumps(r) + "\n")
 
 
 if __name__ == "__main__":

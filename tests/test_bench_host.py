@@ -96,3 +96,25 @@ def test_reference_arm_prints_one_contract_line():
 def test_reference_arm_other_ranks_do_no_work():
     r = _run_reference({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_log_rows_one_per_measured_part(tmp_path):
+    """--log appends the result line, then one JSON row per part (decode,
+    chunked, rooflines, e2e, CPU baseline, each extra and sweep point), each
+    carrying the workload config; a second run appends."""
+    res = {"metric": "m", "value": 1.0, "config": {"workload": "w", "seeds": {"prefill": 1005}},
+           "clocks": {"sm_mhz": 1900.0}, "decode": {"tokens_per_s": 3.0},
+           "chunked": {"tflops": 2.0}, "roofline": {"frac": 0.9}, "e2e": {"value": 0.5},
+           "cpu_baseline": {"value": 0.02, "check_of_timed_output": {"max_abs": 0.01}},
+           "extras": {"a": {"tflops": 4.0}}, "sweep": {"N4096_W1024": {"tflops": 5.0}, "ratio": 2.1}}
+    path = tmp_path / "log.jsonl"
+    bench.write_log(str(path), res)
+    rows = [json.loads(line) for line in path.read_text().splitlines()]
+    assert rows[0] == res
+    parts = [r["part"] for r in rows[1:]]
+    assert parts == ["decode", "chunked", "roofline", "e2e", "cpu_baseline", "extras.a", "sweep.N4096_W1024",
+                     "sweep.ratio"]
+    assert all(r["config"] == res["config"] and r["impl"] == "native" for r in rows[1:])
+    assert rows[-1]["value"] == 2.1 and rows[2]["tflops"] == 2.0
+    bench.write_log(str(path), res)
+    assert len(path.read_text().splitlines()) == 2 * len(rows)
