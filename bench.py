@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
     ap.add_argument("--log", default=None,
                     help="also append the result, and one row per measured part, as JSON lines to this file")
-    ap.add_argument("--ncu-case", choices=["prefill", "prefill_b2", "chunk", "decode"], default=None,
+    ap.add_argument("--ncu-case", choices=["prefill", "prefill_b2", "chunk", "decode", "mixed"], default=None,
                     help="run a reduced case of one kernel three times for an ncu capture (no timing)")
     return ap.parse_args(argv)
 
@@ -714,9 +714,11 @@ def run_ncu_case(case: str) -> None:
     on the device), `prefill` half of it (B=1, same per-unit structure),
     `chunk` the benchmark's chunked prefill (4 x attention + append), `decode`
     a reduced decode (B=16, a quarter of the batch, positions from the same
-    distribution, still above L2).  Prints the algorithmic bytes per launch so
-    a capture's DRAM traffic can be compared with (or scaled to) the
-    benchmark's launch."""
+    distribution, still above L2), `mixed` the benchmark's mixed packed call
+    (4 chunks of 4096 and 60 decode tokens over the decode workload's 1 GB of
+    buffers; its decode tokens run in the decode kernel's cluster mode).
+    Prints the algorithmic bytes per launch so a capture's DRAM traffic can be
+    compared with (or scaled to) the benchmark's launch."""
     import dataclasses
     import torch
     import sliding_window_gqa_prefill_b200 as swa
@@ -749,6 +751,25 @@ def run_ncu_case(case: str) -> None:
               f"the chunk + full K/V buffer), useful FLOPs "
               f"{wl.useful_flops(w.B, w.N, w.W, w.Hq, w.D) - wl.useful_flops(w.B, w.N - w.C, w.W, w.Hq, w.D)}; "
               f"append of {w.C} rows algorithmic bytes {alg_append} (k, v read and written)")
+    elif case == "mixed":
+        import itertools
+        hp, dw = wl.HEADLINE_PREFILL, wl.DECODE_B64
+        d = wl.decode_inputs(dataclasses.replace(dw, steps=1))
+        kc, vc = d["k_cache"].cuda(), d["v_cache"].cuda()
+        lens = [4096] * 4 + [1] * 60
+        total = sum(lens)
+        cu = torch.tensor([0] + list(itertools.accumulate(lens)), dtype=torch.int32, device="cuda")
+        start = d["pos0"].cuda()
+        qm = wl.random_bf16((total, hp.Hq, hp.D), 7001).cuda()
+        km = wl.random_bf16((total, hp.Hkv, hp.D), 7002).cuda()
+        vm = wl.random_bf16((total, hp.Hkv, hp.D), 7003).cuda()
+        om = torch.empty_like(qm)
+        for _ in range(3):
+            swa.swa_prefill_chunk_varlen(qm, km, vm, kc, vc, start, cu, dw.W, hp.scale, out=om)
+        keys = sum(min(int(p) + 1, dw.W) for p in d["pos0"][4:])
+        alg = keys * dw.Hkv * dw.D * 2 * 2 + 60 * hp.Hq * hp.D * 2 * 2
+        print(f"ncu case mixed: decode-token launch algorithmic bytes {alg} (K/V rows in the 60 windows, "
+              f"the own rows included, + q + out rows)")
     else:
         w = dataclasses.replace(wl.DECODE_B64, B=16, steps=1)
         d = wl.decode_inputs(w)
