@@ -437,6 +437,10 @@ def run_native(args):
     e2e_value = weak_scaling_rate(pf_flops * args.steps, world, e2e_ms * 1e-3) / 1e12
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = hout.numel() * 2
+    # the copy bound of that loop: the same bytes moved by plain copies, each
+    # direction alone and both at once (pinned host memory, two streams)
+    pcie = measure_pcie(dev, h2d, d2h, world)
+    pcie["frac_of_both_at_once"] = pcie["both_ms"] / (e2e_ms / args.steps)
 
     # per step: the one-shot prefill, attention + append per chunk, and per
     # decode step the append, the split-KV kernel and the split merge (the
@@ -521,7 +525,7 @@ def run_native(args):
                         "ms": ch_total / args.steps,
                         "frac": chunk_tflops / world / peaks["bf16"]},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps, "copy_bound": pcie},
             "extras": extras,
             "sweep": sweep,
             "gpu_launches": launches_per_step * args.steps,
@@ -535,6 +539,35 @@ def run_native(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return result
+
+
+def measure_pcie(dev, h2d_bytes: int, d2h_bytes: int, world: int) -> dict:
+    """Plain copies of the end-to-end step's bytes between pinned host memory
+    and the device: host->device alone, device->host alone, and both at once
+    on two streams (median of 5 each, CUDA events, max over ranks)."""
+    import torch
+    hin = torch.empty(h2d_bytes, dtype=torch.uint8, pin_memory=True)
+    din = torch.empty(h2d_bytes, dtype=torch.uint8, device=dev)
+    dout = torch.empty(d2h_bytes, dtype=torch.uint8, device=dev)
+    hout = torch.empty(d2h_bytes, dtype=torch.uint8, pin_memory=True)
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+
+    def both():
+        s1.wait_stream(cur)
+        s2.wait_stream(cur)
+        with torch.cuda.stream(s1):
+            din.copy_(hin, non_blocking=True)
+        with torch.cuda.stream(s2):
+            hout.copy_(dout, non_blocking=True)
+        cur.wait_stream(s1)
+        cur.wait_stream(s2)
+
+    t_in = max_over_ranks(_time_ms(lambda: din.copy_(hin, non_blocking=True), 5), world)
+    t_out = max_over_ranks(_time_ms(lambda: hout.copy_(dout, non_blocking=True), 5), world)
+    t_both = max_over_ranks(_time_ms(both, 5), world)
+    return {"h2d_gbs": h2d_bytes / t_in / 1e6, "d2h_gbs": d2h_bytes / t_out / 1e6, "both_ms": t_both,
+            "note": "frac_of_both_at_once = time of the step's bytes copied both ways at once / e2e time per step"}
 
 
 def _time_ms(fn, iters: int) -> float:
