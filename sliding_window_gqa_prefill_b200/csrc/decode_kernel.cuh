@@ -29,6 +29,11 @@
 //    most blocks take no maximum.
 //  * warps and splits are merged by log-sum-exp: in shared memory inside a
 //    block, and by swa_decode_combine_kernel across splits.
+//  * the one-token sequences of a packed chunk batch (decode steps in a
+//    mixed pre-fill call) take a third mode: the token's own K/V come from
+//    its packed row (the buffer is written after the attention), and the 4
+//    splits of a window are the blocks of one cluster, merged through
+//    distributed shared memory instead of a workspace.
 #pragma once
 
 #include "device_common.cuh"
