@@ -142,7 +142,10 @@ swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
                         int D, int W, float scale, void *workspace,
                         size_t workspace_bytes, swa_stream_t stream);
 
-/* Workspace bytes swa_decode needs for these sizes (0 if they are invalid). */
+/* Workspace bytes swa_decode needs for these sizes (0 if they are invalid).
+ * The window is cut into splits of up to 1024 keys, smaller (down to 256)
+ * when B * Hkv is small, so that a small batch still spreads over the GPU;
+ * the split length, and so this size, depends on B, Hkv and W only. */
 size_t swa_decode_workspace_size(int B, int Hq, int Hkv, int D, int W);
 
 /*

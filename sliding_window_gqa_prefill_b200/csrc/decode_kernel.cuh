@@ -40,7 +40,11 @@
 
 namespace swa {
 
-constexpr int kDecodeSplit = 1024;     // keys per block (1024 measured 0.5-2.5% faster than 512)
+// keys per block: at most kDecodeSplit (1024 measured 0.5-2.5% faster than
+// 512 at B=64), fewer (down to kDecodeMinSplit) for batches too small to fill
+// the GPU; the host picks it per launch from the sizes alone
+constexpr int kDecodeSplit = 1024;
+constexpr int kDecodeMinSplit = 256;
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeBlk = 16;         // keys per tensor-core block
 constexpr int kDecodeStages = 3;       // per-warp ring depth, in 16-key blocks
@@ -138,7 +142,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                   float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2,
                   int rope, const RopeTable rope_freq, const __nv_bfloat16 *__restrict__ ksink,
                   const __nv_bfloat16 *__restrict__ vsink, int S, const int32_t *__restrict__ cu,
-                  int total) {
+                  int total, int split_len) {
     constexpr bool SINKS = MODE == kDecodeSinks;
     using Cfg = DecodeCfg<D, G>;
     constexpr int CH = Cfg::CH, RB = Cfg::ROW_BYTES;
@@ -170,7 +174,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const int L = Lw + ns;
     constexpr int kClusterKeys = kDecodeClusterSplits * kDecodeBlk;
     const int split_keys =
-        (MODE == kDecodePackedRows) ? (L + kClusterKeys - 1) / kClusterKeys * kDecodeBlk : kDecodeSplit;
+        (MODE == kDecodePackedRows) ? (L + kClusterKeys - 1) / kClusterKeys * kDecodeBlk : split_len;
     // MODE 2: a block past the window's keys still takes part in the merge
     if (MODE != kDecodePackedRows && split * split_keys >= L) return;
     const int begin = min(split * split_keys, L);
@@ -428,14 +432,14 @@ template <int D, int G>
 __global__ void __launch_bounds__(1024)
 swa_decode_combine_kernel(const int32_t *__restrict__ pos, const float2 *__restrict__ ws_ml,
                           const float *__restrict__ ws_o, __nv_bfloat16 *__restrict__ out,
-                          int Hkv, int W, int nsplit_max, int S) {
+                          int Hkv, int W, int nsplit_max, int S, int split_len) {
     const int g = blockIdx.x, b = blockIdx.y;
     const int Hq = Hkv * G;
     const int p = __ldg(pos + b);
     if (p < 0) return;
     const int ns = (S > 0 && p >= W) ? min(S, p - W + 1) : 0;
     const int L = ((p >= W - 1) ? W : p + 1) + ns;
-    const int nsplit = (L + kDecodeSplit - 1) / kDecodeSplit;
+    const int nsplit = (L + split_len - 1) / split_len;
     if (nsplit <= 1 || !in_bounds(nsplit - 1, nsplit_max)) return;
     const size_t base = (size_t)(b * Hkv + g) * nsplit_max;
     constexpr int kUnrolled = 16;            // splits loaded side by side (W <= 8192)

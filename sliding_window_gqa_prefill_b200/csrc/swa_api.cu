@@ -172,14 +172,32 @@ swa_status_t launch_append(const void *k_new, const void *v_new, void *k_cache, 
     return SWA_OK;
 }
 
-int decode_nsplit_max(int W) { return (W + swa::kDecodeSplit - 1) / swa::kDecodeSplit; }
+// Keys per decode split for a launch over L = W (+ S) keys: kDecodeSplit, or
+// fewer (multiples of 64, at least kDecodeMinSplit) when B * Hkv windows of
+// kDecodeSplit keys would give fewer than ~256 blocks, so that a small batch
+// still spreads over the GPU.  A function of the sizes only: the workspace
+// size follows from it.
+int decode_split_keys(int B, int Hkv, int L) {
+    const long long pairs = (long long)B * Hkv;
+    const long long want = (256 + pairs - 1) / pairs;       // splits per (sequence, kv head)
+    long long split = ((L + want - 1) / want + 63) / 64 * 64;
+    if (split < swa::kDecodeMinSplit) split = swa::kDecodeMinSplit;
+    if (split > swa::kDecodeSplit) split = swa::kDecodeSplit;
+    return (int)split;
+}
+
+int decode_nsplit_max(int B, int Hkv, int L) {
+    const int split = decode_split_keys(B, Hkv, L);
+    return (int)(((long long)L + split - 1) / split);
+}
 
 template <int D, int G>
 swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, const int32_t *pos,
                               void *out, int B, int Hkv, int W, float scale, void *ws,
                               const swa::RopeTable *rope, cudaStream_t s, const void *ksink,
                               const void *vsink, int S) {
-    const int nsm = decode_nsplit_max(W + S);
+    const int nsm = decode_nsplit_max(B, Hkv, W + S);
+    const int split = decode_split_keys(B, Hkv, W + S);
     const size_t o_elems = (size_t)B * Hkv * nsm * G * D;
     float *ws_o = static_cast<float *>(ws);
     float2 *ws_ml = ws ? reinterpret_cast<float2 *>(static_cast<char *>(ws) + ((o_elems * 4 + 255) & ~size_t(255)))
@@ -192,11 +210,11 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
         static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
         Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{},
         static_cast<const __nv_bfloat16 *>(ksink), static_cast<const __nv_bfloat16 *>(vsink), S,
-        nullptr, 0);
+        nullptr, 0, split);
     SWA_CUDA_TRY(cudaGetLastError());
     if (nsm > 1) {
         swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), G * D, 0, s>>>(
-            pos, ws_ml, ws_o, static_cast<__nv_bfloat16 *>(out), Hkv, W, nsm, S);
+            pos, ws_ml, ws_o, static_cast<__nv_bfloat16 *>(out), Hkv, W, nsm, S, split);
         SWA_CUDA_TRY(cudaGetLastError());
     }
     return SWA_OK;
@@ -246,7 +264,7 @@ swa_status_t launch_decode_packed_dg(const void *q, const void *k, const void *v
     float *no_o = nullptr;
     SWA_CUDA_TRY(cudaLaunchKernelEx(&cfg, swa::swa_decode_kernel<D, G, swa::kDecodePackedRows>, qb, kcb, vcb,
                                     start_pos, ob, no_ml, no_o, Hkv, W, 1, scale * kLog2e, 0, swa::RopeTable{},
-                                    kb, vb, 0, cu, total));
+                                    kb, vb, 0, cu, total, 0));
     return SWA_OK;
 }
 
@@ -485,7 +503,7 @@ swa_status_t append_impl(const void *k_new, const void *v_new, void *k_cache, vo
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
     if (B < 1 || W < 1 || check_heads(Hq, Hkv, D) != SWA_OK) return 0;
-    const size_t nsm = (size_t)decode_nsplit_max(W);
+    const size_t nsm = (size_t)decode_nsplit_max(B, Hkv, W);
     const size_t rows = (size_t)B * Hq * nsm;        // (b, kv head, split, head in group)
     const size_t o_bytes = (rows * D * 4 + 255) & ~size_t(255);
     return o_bytes + rows * 8;
@@ -520,7 +538,7 @@ swa_status_t decode_impl(const void *q, const void *k_cache, const void *v_cache
                          const swa::RopeTable *rope, cudaStream_t s) {
     if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
     const size_t need = decode_workspace_bytes(B, Hq, Hkv, D, W);
-    if (decode_nsplit_max(W) > 1) {
+    if (decode_nsplit_max(B, Hkv, W) > 1) {
         if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
     }
@@ -690,7 +708,7 @@ swa_status_t swa_decode_sinks(const void *q, const void *k_cache, const void *v_
     if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
     if ((long long)W + S > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
     const size_t need = decode_workspace_bytes(B, Hq, Hkv, D, W + S);
-    if (decode_nsplit_max(W + S) > 1) {
+    if (decode_nsplit_max(B, Hkv, W + S) > 1) {
         if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
     }

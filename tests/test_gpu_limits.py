@@ -63,8 +63,9 @@ def _filled_buffers(oracle_mod, B, W, Hkv, D, counts, seed):
 
 @pytest.mark.parametrize("W,Hq,Hkv,D", [(20000, 8, 2, 128), (32768, 8, 2, 64), (20000, 4, 4, 128)])
 def test_decode_beyond_16_splits(oracle_mod, W, Hq, Hkv, D):
-    """20 and 32 splits of 1024 keys: the merge takes its looped path; the
-    static-scratch entry point gives the same bits."""
+    """21 to 43 splits (B=3 is a small batch: splits of 512-960 keys): the
+    merge takes its looped path; the static-scratch entry point gives the
+    same bits."""
     B = 3
     pos = np.array([W - 2, W + 5, 3 * W + 17], np.int32)
     kr, vr, sp = _filled_buffers(oracle_mod, B, W, Hkv, D, pos, 4000 + W)   # positions 0 .. pos-1

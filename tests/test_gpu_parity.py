@@ -241,8 +241,8 @@ def _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps, seed):
     (2, 4, 4, 64, 700, [10, 2000]),                     # G=1, W not a multiple of 16 keys per block
     (2, 16, 2, 128, 1000, [999, 5]),                    # G=8
     (2, 4, 2, 64, 300, [299, 77]),                      # G=2, single split
-    (2, 8, 2, 128, 8192, [8191, 20000]),                # 8 splits: workspace merge path
-    (1, 4, 1, 64, 5000, [4999]),                        # 5 splits, the last one partial, G=4, D=64
+    (2, 8, 2, 128, 8192, [8191, 20000]),                # small batch: 32 splits of 256 keys, merged
+    (1, 4, 1, 64, 5000, [4999]),                        # 20 splits of 256, the last one partial, G=4, D=64
 ])
 def test_decode_edge_cases(oracle_mod, B, Hq, Hkv, D, W, pos0):
     _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps=3, seed=B * W + D)

@@ -69,7 +69,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     swa.build()
     L = swa.lib()
-    B, Hq, Hkv, D, W = 256, 32, 8, 128, 8192          # needs ~68 MB of partials
+    B, Hq, Hkv, D, W = 256, 32, 8, 128, 8192          # needs ~34 MB of partials
     assert swa.swa_decode_workspace_size(B, Hq, Hkv, D, W) > (16 << 20)
     st = L.swa_decode_noalloc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, B, Hq, Hkv, D, W, 0.1, None)
     assert st == swa.SWA_ERR_UNSUPPORTED
