@@ -70,7 +70,7 @@ struct DecodeCfg {
     static constexpr int MERGE_BYTES = (kDecodeWarps + 1) * G * (D + 2) * 4;
     static constexpr int SMEM_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
     static_assert(D == 64 || D == 128, "head_dim");
-    static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "group size 1, 2, 4 or 8");
+    static_assert(G >= 1 && G <= 8, "group size 1 to 8 (the rows 0..7 of the MMA tile)");
     static_assert(CPL * 32 == kDecodeBlk * CH, "copies per lane");
 };
 

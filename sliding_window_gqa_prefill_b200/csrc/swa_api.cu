@@ -106,9 +106,12 @@ swa_status_t device_info(DeviceInfo **out) {
     SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, swa::kDecodePackedRows>, \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,           \
                                       swa::DecodeCfg<DD, GG>::SMEM_BYTES));
-        SWA_SET_DECODE_ATTR(64, 1) SWA_SET_DECODE_ATTR(64, 2) SWA_SET_DECODE_ATTR(64, 4)
-        SWA_SET_DECODE_ATTR(64, 8) SWA_SET_DECODE_ATTR(128, 1) SWA_SET_DECODE_ATTR(128, 2)
-        SWA_SET_DECODE_ATTR(128, 4) SWA_SET_DECODE_ATTR(128, 8)
+        SWA_SET_DECODE_ATTR(64, 1) SWA_SET_DECODE_ATTR(64, 2) SWA_SET_DECODE_ATTR(64, 3)
+        SWA_SET_DECODE_ATTR(64, 4) SWA_SET_DECODE_ATTR(64, 5) SWA_SET_DECODE_ATTR(64, 6)
+        SWA_SET_DECODE_ATTR(64, 7) SWA_SET_DECODE_ATTR(64, 8)
+        SWA_SET_DECODE_ATTR(128, 1) SWA_SET_DECODE_ATTR(128, 2) SWA_SET_DECODE_ATTR(128, 3)
+        SWA_SET_DECODE_ATTR(128, 4) SWA_SET_DECODE_ATTR(128, 5) SWA_SET_DECODE_ATTR(128, 6)
+        SWA_SET_DECODE_ATTR(128, 7) SWA_SET_DECODE_ATTR(128, 8)
 #undef SWA_SET_DECODE_ATTR
         d.attrs_set = true;
     }
@@ -228,7 +231,11 @@ swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *v
     switch (G) {
         case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 3: return launch_decode_dg<D, 3>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 5: return launch_decode_dg<D, 5>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 6: return launch_decode_dg<D, 6>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 7: return launch_decode_dg<D, 7>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
         default: return SWA_ERR_UNSUPPORTED;
     }
@@ -276,7 +283,11 @@ bool launch_decode_packed_d(int G, swa_status_t *e, const void *q, const void *k
     switch (G) {
         case 1: *e = launch_decode_packed_dg<D, 1>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
         case 2: *e = launch_decode_packed_dg<D, 2>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 3: *e = launch_decode_packed_dg<D, 3>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
         case 4: *e = launch_decode_packed_dg<D, 4>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 5: *e = launch_decode_packed_dg<D, 5>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 6: *e = launch_decode_packed_dg<D, 6>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 7: *e = launch_decode_packed_dg<D, 7>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
         case 8: *e = launch_decode_packed_dg<D, 8>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
         default: return false;
     }

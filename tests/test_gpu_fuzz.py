@@ -121,6 +121,40 @@ def test_fuzz_decode(oracle_mod, case):
     assert np.array_equal(f64(kg.cpu()), kr) and np.array_equal(f64(vg.cpu()), vr)
 
 
+@pytest.mark.parametrize("G", range(1, 9))
+def test_fuzz_decode_every_group_size(oracle_mod, G):
+    """Decode at each group size 1-8 (odd ones included: rows G..15 of the MMA
+    tile are zero), with and without RoPE, random shapes and positions."""
+    rng = np.random.default_rng(12400 + G)
+    B = int(rng.integers(1, 5))
+    W = int(rng.integers(8, 3000))
+    Hkv = int(rng.choice([1, 2, 3]))
+    Hq, D = Hkv * G, int(rng.choice([64, 128]))
+    seed = 12500 + 10 * G
+    kc = wl.random_bf16((B, W, Hkv, D), seed)
+    vc = wl.random_bf16((B, W, Hkv, D), seed + 1)
+    pos0 = rng.integers(0, 3 * W, size=B).astype(np.int32)
+    sp = oracle_mod.slot_positions(pos0, W)
+    kr, vr = f64(kc), f64(vc)
+    kg, vg = kc.cuda(), vc.cuda()
+    scale = 1.0 / math.sqrt(D)
+    for s in range(2):
+        q = wl.random_bf16((B, Hq, D), seed + 10 + s)
+        kn = wl.random_bf16((B, 1, Hkv, D), seed + 20 + s)
+        vn = wl.random_bf16((B, 1, Hkv, D), seed + 30 + s)
+        pos = torch.from_numpy(pos0 + s)
+        swa.swa_cache_append(kn.cuda(), vn.cuda(), kg, vg, pos.cuda())
+        out = swa.swa_decode(q.cuda(), kg, vg, pos.cuda(), scale)
+        out_r = swa.swa_decode(q.cuda(), kg, vg, pos.cuda(), scale, rope_theta=10000.0)
+        torch.cuda.synchronize()
+        oracle_mod.cache_append(kr, vr, sp, f64(kn), f64(vn), pos.numpy())
+        ref = oracle_mod.swa_decode(f64(q), kr, vr, sp, pos.numpy(), W, scale)
+        close(out.cpu(), ref, f"decode G={G} B{B} W{W} D{D} step {s}")
+        qr = oracle_mod.rope(f64(q)[:, None], pos.numpy(), 10000.0)[:, 0]
+        close(out_r.cpu(), oracle_mod.swa_decode(qr, kr, vr, sp, pos.numpy(), W, scale), f"decode RoPE G={G} step {s}")
+    assert np.array_equal(f64(kg.cpu()), kr) and np.array_equal(f64(vg.cpu()), vr)
+
+
 @pytest.mark.parametrize("case", range(6))
 def test_fuzz_varlen(oracle_mod, case):
     """Packed batch of random lengths (zeros included): each sequence equals its own one-shot prefill."""
