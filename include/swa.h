@@ -129,10 +129,12 @@ swa_status_t swa_cache_append(const void *k_new, const void *v_new,
  *   pos : int32 [B] device array, position of the new token, whose K/V must
  *         already be in the cache (swa_cache_append first).
  * Each sequence reads slots 0 .. min(pos[b]+1, W)-1; softmax is order-free,
- * so the wrap needs no reordering.  Group sizes Hq/Hkv of 1 to 8 are covered
- * (Mistral-7B: 4); larger ones return SWA_ERR_UNSUPPORTED, as do the _rope,
- * _sinks and _noalloc forms.  (A decode step of any group size runs through
- * swa_prefill_chunk_varlen as a length-1 sequence.)
+ * so the wrap needs no reordering.  Any group size Hq/Hkv (Mistral-7B: 4): the
+ * query heads of a group are the rows of a tensor-core tile, up to 8 at a
+ * time, so a group of G heads runs as G / Gt groups of Gt heads (Gt the
+ * largest divisor of G up to 8), each reading the K/V head again; the same
+ * holds for the _rope, _sinks and _noalloc forms.  Hkv * G / Gt above 65535
+ * returns SWA_ERR_UNSUPPORTED.
  * workspace: device scratch of at least swa_decode_workspace_size() bytes,
  *   256-byte aligned, owned by the caller; its contents need no set-up and are
  *   overwritten.  Calls that share a workspace must not overlap on the GPU.
@@ -204,10 +206,9 @@ swa_status_t swa_prefill_varlen(const void *q, const void *k, const void *v, voi
  * its own key and the W-1 positions before it), so pre-fill chunks and decode
  * tokens share one call.  Any length is accepted: a sequence longer than W
  * leaves its last W positions in the buffer.  Attend first, then write.
- * With group sizes Hq/Hkv of 1 to 8 the length-1 sequences are computed by
- * the decode kernel (reading their own key and value from the packed k/v
- * rows) and the others by the prefill kernel; with larger group sizes the
- * prefill kernel takes them all.  Up to three kernels on `stream`. */
+ * The length-1 sequences are computed by the decode kernel (reading their
+ * own key and value from the packed k/v rows, heads taken as in swa_decode)
+ * and the others by the prefill kernel.  Up to three kernels on `stream`. */
 swa_status_t swa_prefill_chunk_varlen(const void *q, const void *k, const void *v, void *k_cache,
                                       void *v_cache, const int32_t *start_pos,
                                       const int32_t *cu_seqlens, void *out, int B, int total,

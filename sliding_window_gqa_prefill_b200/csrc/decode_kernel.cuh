@@ -142,7 +142,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                   float *__restrict__ ws_o, int Hkv, int W, int nsplit_max, float scale_log2,
                   int rope, const RopeTable rope_freq, const __nv_bfloat16 *__restrict__ ksink,
                   const __nv_bfloat16 *__restrict__ vsink, int S, const int32_t *__restrict__ cu,
-                  int total, int split_len) {
+                  int total, int split_len, int kv_rep) {
     constexpr bool SINKS = MODE == kDecodeSinks;
     using Cfg = DecodeCfg<D, G>;
     constexpr int CH = Cfg::CH, RB = Cfg::ROW_BYTES;
@@ -208,13 +208,17 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             }
     }
 
-    const size_t row_stride = (size_t)Hkv * D;     // elements between consecutive slots
-    const __nv_bfloat16 *kbase = kc + ((size_t)b * W * Hkv + g) * D;
-    const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv + g) * D;
-    const __nv_bfloat16 *ksbase = ns ? ksink + ((size_t)b * S * Hkv + g) * D : kbase;
-    const __nv_bfloat16 *vsbase = ns ? vsink + ((size_t)b * S * Hkv + g) * D : vbase;
-    const __nv_bfloat16 *knew = (MODE == kDecodePackedRows) ? ksink + ((size_t)qrow * Hkv + g) * D : kbase;
-    const __nv_bfloat16 *vnew = (MODE == kDecodePackedRows) ? vsink + ((size_t)qrow * Hkv + g) * D : vbase;
+    // K/V heads in memory: a group of more than 8 query heads (or one with no
+    // divisor up to 8 above 1) is taken as kv_rep groups of G heads, all
+    // reading K/V head g / kv_rep (Hkv counts those groups)
+    const int Hkv_mem = Hkv / kv_rep, gk = g / kv_rep;
+    const size_t row_stride = (size_t)Hkv_mem * D;  // elements between consecutive slots
+    const __nv_bfloat16 *kbase = kc + ((size_t)b * W * Hkv_mem + gk) * D;
+    const __nv_bfloat16 *vbase = vc + ((size_t)b * W * Hkv_mem + gk) * D;
+    const __nv_bfloat16 *ksbase = ns ? ksink + ((size_t)b * S * Hkv_mem + gk) * D : kbase;
+    const __nv_bfloat16 *vsbase = ns ? vsink + ((size_t)b * S * Hkv_mem + gk) * D : vbase;
+    const __nv_bfloat16 *knew = (MODE == kDecodePackedRows) ? ksink + ((size_t)qrow * Hkv_mem + gk) * D : kbase;
+    const __nv_bfloat16 *vnew = (MODE == kDecodePackedRows) ? vsink + ((size_t)qrow * Hkv_mem + gk) * D : vbase;
 
     const int nblk = (end - begin + kDecodeBlk - 1) / kDecodeBlk;
     const int my_blocks = (nblk > warp) ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;

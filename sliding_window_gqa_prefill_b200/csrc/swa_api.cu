@@ -189,16 +189,29 @@ int decode_split_keys(int B, int Hkv, int L) {
     return (int)split;
 }
 
+// The decode kernel takes the Hq/Hkv query heads that share a K/V head as
+// the rows of its MMA tile, at most 8 at a time: a group of G heads runs as
+// rep = G / Gt groups of Gt heads, Gt the largest divisor of G up to 8 (each
+// K/V head then read rep times).  Returns Gt.
+int decode_group(int Hq, int Hkv, int *rep) {
+    const int G = Hq / Hkv;
+    int gt = G < 8 ? G : 8;
+    while (G % gt != 0) --gt;
+    *rep = G / gt;
+    return gt;
+}
+
 int decode_nsplit_max(int B, int Hkv, int L) {
     const int split = decode_split_keys(B, Hkv, L);
     return (int)(((long long)L + split - 1) / split);
 }
 
+// Hkv: groups of G query heads (kv_rep groups per K/V head in memory).
 template <int D, int G>
 swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, const int32_t *pos,
                               void *out, int B, int Hkv, int W, float scale, void *ws,
                               const swa::RopeTable *rope, cudaStream_t s, const void *ksink,
-                              const void *vsink, int S) {
+                              const void *vsink, int S, int kv_rep) {
     const int nsm = decode_nsplit_max(B, Hkv, W + S);
     const int split = decode_split_keys(B, Hkv, W + S);
     const size_t o_elems = (size_t)B * Hkv * nsm * G * D;
@@ -213,7 +226,7 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
         static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out), ws_ml, ws_o,
         Hkv, W, nsm, scale * kLog2e, rope ? 1 : 0, rope ? *rope : swa::RopeTable{},
         static_cast<const __nv_bfloat16 *>(ksink), static_cast<const __nv_bfloat16 *>(vsink), S,
-        nullptr, 0, split);
+        nullptr, 0, split, kv_rep);
     SWA_CUDA_TRY(cudaGetLastError());
     if (nsm > 1) {
         swa::swa_decode_combine_kernel<D, G><<<dim3(Hkv, B), G * D, 0, s>>>(
@@ -224,19 +237,19 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
 }
 
 template <int D>
-swa_status_t launch_decode_d(int G, const void *q, const void *kc, const void *vc,
+swa_status_t launch_decode_d(int G, int kv_rep, const void *q, const void *kc, const void *vc,
                              const int32_t *pos, void *out, int B, int Hkv, int W, float scale,
                              void *ws, const swa::RopeTable *rope, cudaStream_t s,
                              const void *ksink = nullptr, const void *vsink = nullptr, int S = 0) {
     switch (G) {
-        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 3: return launch_decode_dg<D, 3>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 5: return launch_decode_dg<D, 5>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 6: return launch_decode_dg<D, 6>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 7: return launch_decode_dg<D, 7>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
-        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S);
+        case 1: return launch_decode_dg<D, 1>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 2: return launch_decode_dg<D, 2>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 3: return launch_decode_dg<D, 3>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 4: return launch_decode_dg<D, 4>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 5: return launch_decode_dg<D, 5>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 6: return launch_decode_dg<D, 6>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 7: return launch_decode_dg<D, 7>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
+        case 8: return launch_decode_dg<D, 8>(q, kc, vc, pos, out, B, Hkv, W, scale, ws, rope, s, ksink, vsink, S, kv_rep);
         default: return SWA_ERR_UNSUPPORTED;
     }
 }
@@ -248,7 +261,7 @@ template <int D, int G>
 swa_status_t launch_decode_packed_dg(const void *q, const void *k, const void *v, const void *kc,
                                      const void *vc, const int32_t *start_pos, const int32_t *cu,
                                      void *out, int B, int total, int Hkv, int W, float scale,
-                                     cudaStream_t s) {
+                                     cudaStream_t s, int kv_rep) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(swa::kDecodeClusterSplits, Hkv, B);
     cfg.blockDim = dim3(swa::kDecodeWarps * 32);
@@ -271,24 +284,24 @@ swa_status_t launch_decode_packed_dg(const void *q, const void *k, const void *v
     float *no_o = nullptr;
     SWA_CUDA_TRY(cudaLaunchKernelEx(&cfg, swa::swa_decode_kernel<D, G, swa::kDecodePackedRows>, qb, kcb, vcb,
                                     start_pos, ob, no_ml, no_o, Hkv, W, 1, scale * kLog2e, 0, swa::RopeTable{},
-                                    kb, vb, 0, cu, total, 0));
+                                    kb, vb, 0, cu, total, 0, kv_rep));
     return SWA_OK;
 }
 
 // false when the decode kernel has no instance for this head group
 template <int D>
-bool launch_decode_packed_d(int G, swa_status_t *e, const void *q, const void *k, const void *v,
+bool launch_decode_packed_d(int G, int kv_rep, swa_status_t *e, const void *q, const void *k, const void *v,
                             const void *kc, const void *vc, const int32_t *start_pos, const int32_t *cu,
                             void *out, int B, int total, int Hkv, int W, float scale, cudaStream_t s) {
     switch (G) {
-        case 1: *e = launch_decode_packed_dg<D, 1>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 2: *e = launch_decode_packed_dg<D, 2>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 3: *e = launch_decode_packed_dg<D, 3>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 4: *e = launch_decode_packed_dg<D, 4>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 5: *e = launch_decode_packed_dg<D, 5>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 6: *e = launch_decode_packed_dg<D, 6>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 7: *e = launch_decode_packed_dg<D, 7>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
-        case 8: *e = launch_decode_packed_dg<D, 8>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s); return true;
+        case 1: *e = launch_decode_packed_dg<D, 1>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 2: *e = launch_decode_packed_dg<D, 2>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 3: *e = launch_decode_packed_dg<D, 3>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 4: *e = launch_decode_packed_dg<D, 4>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 5: *e = launch_decode_packed_dg<D, 5>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 6: *e = launch_decode_packed_dg<D, 6>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 7: *e = launch_decode_packed_dg<D, 7>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
+        case 8: *e = launch_decode_packed_dg<D, 8>(q, k, v, kc, vc, start_pos, cu, out, B, total, Hkv, W, scale, s, kv_rep); return true;
         default: return false;
     }
 }
@@ -474,10 +487,15 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
         // length-1 sequences (decode tokens) go to the decode kernel, which
         // reads their windows at memory speed instead of as 128-row tiles
         swa_status_t ed = SWA_OK;
-        const bool dec = D == 128 ? launch_decode_packed_d<128>(G, &ed, q, k, v, k_cache, v_cache, start_pos,
-                                                                cu_seqlens, out, B, C, Hkv, W, scale, s)
-                                  : launch_decode_packed_d<64>(G, &ed, q, k, v, k_cache, v_cache, start_pos,
-                                                               cu_seqlens, out, B, C, Hkv, W, scale, s);
+        int rep = 1;
+        const int gt = decode_group(Hq, Hkv, &rep);
+        const bool fits = (long long)Hkv * rep <= 65535;
+        const bool dec = fits && (D == 128 ? launch_decode_packed_d<128>(gt, rep, &ed, q, k, v, k_cache, v_cache,
+                                                                         start_pos, cu_seqlens, out, B, C, Hkv * rep,
+                                                                         W, scale, s)
+                                           : launch_decode_packed_d<64>(gt, rep, &ed, q, k, v, k_cache, v_cache,
+                                                                        start_pos, cu_seqlens, out, B, C, Hkv * rep,
+                                                                        W, scale, s));
         if (ed) return ed;
         p.skip_len1 = dec ? 1 : 0;
     }
@@ -514,7 +532,10 @@ swa_status_t append_impl(const void *k_new, const void *v_new, void *k_cache, vo
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
     if (B < 1 || W < 1 || check_heads(Hq, Hkv, D) != SWA_OK) return 0;
-    const size_t nsm = (size_t)decode_nsplit_max(B, Hkv, W);
+    int rep = 1;
+    decode_group(Hq, Hkv, &rep);
+    if ((long long)Hkv * rep > 65535) return 0;
+    const size_t nsm = (size_t)decode_nsplit_max(B, Hkv * rep, W);
     const size_t rows = (size_t)B * Hq * nsm;        // (b, kv head, split, head in group)
     const size_t o_bytes = (rows * D * 4 + 255) & ~size_t(255);
     return o_bytes + rows * 8;
@@ -529,18 +550,23 @@ swa_status_t decode_checks(const void *q, const void *k_cache, const void *v_cac
         return SWA_ERR_INVALID_ARG;
     if (B < 1 || W < 1 || bad_scale(scale)) return SWA_ERR_INVALID_ARG;
     if (swa_status_t e = check_heads(Hq, Hkv, D)) return e;
-    if (B > 65535 || Hkv > 65535) return SWA_ERR_UNSUPPORTED;
+    int rep = 1;
+    decode_group(Hq, Hkv, &rep);
+    if (B > 65535 || (long long)Hkv * rep > 65535) return SWA_ERR_UNSUPPORTED;
     return SWA_OK;
 }
 
 swa_status_t decode_launch(const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *pos, void *out, int B, int Hq, int Hkv, int D, int W,
                            float scale, void *workspace, const swa::RopeTable *rope, cudaStream_t s) {
-    const int G = Hq / Hkv;
+    int rep = 1;
+    const int G = decode_group(Hq, Hkv, &rep);
     DeviceInfo *dev = nullptr;
     if (swa_status_t e = device_info(&dev)) return e;
-    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, rope, s)
-                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, rope, s);
+    return D == 128 ? launch_decode_d<128>(G, rep, q, k_cache, v_cache, pos, out, B, Hkv * rep, W, scale, workspace,
+                                           rope, s)
+                    : launch_decode_d<64>(G, rep, q, k_cache, v_cache, pos, out, B, Hkv * rep, W, scale, workspace,
+                                          rope, s);
 }
 
 swa_status_t decode_impl(const void *q, const void *k_cache, const void *v_cache,
@@ -549,7 +575,9 @@ swa_status_t decode_impl(const void *q, const void *k_cache, const void *v_cache
                          const swa::RopeTable *rope, cudaStream_t s) {
     if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
     const size_t need = decode_workspace_bytes(B, Hq, Hkv, D, W);
-    if (decode_nsplit_max(B, Hkv, W) > 1) {
+    int rep = 1;
+    decode_group(Hq, Hkv, &rep);
+    if (decode_nsplit_max(B, Hkv * rep, W) > 1) {
         if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
     }
@@ -719,18 +747,19 @@ swa_status_t swa_decode_sinks(const void *q, const void *k_cache, const void *v_
     if (swa_status_t e = decode_checks(q, k_cache, v_cache, pos, out, B, Hq, Hkv, D, W, scale)) return e;
     if ((long long)W + S > 0x7fffffffll) return SWA_ERR_UNSUPPORTED;
     const size_t need = decode_workspace_bytes(B, Hq, Hkv, D, W + S);
-    if (decode_nsplit_max(B, Hkv, W + S) > 1) {
+    int rep = 1;
+    const int G = decode_group(Hq, Hkv, &rep);
+    if (decode_nsplit_max(B, Hkv * rep, W + S) > 1) {
         if (!workspace || workspace_bytes < need) return SWA_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SWA_ERR_INVALID_ARG;
     }
     DeviceInfo *dev = nullptr;
     if (swa_status_t e = device_info(&dev)) return e;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int G = Hq / Hkv;
-    return D == 128 ? launch_decode_d<128>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, nullptr, s,
-                                           k_sink, v_sink, S)
-                    : launch_decode_d<64>(G, q, k_cache, v_cache, pos, out, B, Hkv, W, scale, workspace, nullptr, s,
-                                          k_sink, v_sink, S);
+    return D == 128 ? launch_decode_d<128>(G, rep, q, k_cache, v_cache, pos, out, B, Hkv * rep, W, scale, workspace,
+                                           nullptr, s, k_sink, v_sink, S)
+                    : launch_decode_d<64>(G, rep, q, k_cache, v_cache, pos, out, B, Hkv * rep, W, scale, workspace,
+                                          nullptr, s, k_sink, v_sink, S);
 }
 
 swa_status_t swa_get_device_status(swa_stream_t stream) {

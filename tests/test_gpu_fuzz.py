@@ -121,10 +121,12 @@ def test_fuzz_decode(oracle_mod, case):
     assert np.array_equal(f64(kg.cpu()), kr) and np.array_equal(f64(vg.cpu()), vr)
 
 
-@pytest.mark.parametrize("G", range(1, 9))
+@pytest.mark.parametrize("G", list(range(1, 10)) + [11, 12, 16])
 def test_fuzz_decode_every_group_size(oracle_mod, G):
-    """Decode at each group size 1-8 (odd ones included: rows G..15 of the MMA
-    tile are zero), with and without RoPE, random shapes and positions."""
+    """Decode at each group size 1-9 and at 11, 12 and 16 (odd ones included:
+    rows past the group in the MMA tile are zero; groups above 8 run as
+    several groups of up to 8 heads on the same K/V head, 11 as 11 groups of
+    one), with and without RoPE, random shapes and positions."""
     rng = np.random.default_rng(12400 + G)
     B = int(rng.integers(1, 5))
     W = int(rng.integers(8, 3000))

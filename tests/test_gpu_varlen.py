@@ -2,8 +2,8 @@
 sequence: packed one-shot prefill, and mixed calls in which some sequences
 pre-fill a chunk (through their rolling buffer), some decode one token, one
 chunk is longer than the window and one sequence is empty.  The one-token
-sequences go to the decode kernel for group sizes 1 to 8 and stay in the
-attention kernel for larger ones (16 here); both are checked."""
+sequences go to the decode kernel (group sizes above 8 as several groups of
+up to 8 heads on the same K/V head, 16 here)."""
 import math
 
 import numpy as np
@@ -107,12 +107,12 @@ def test_mixed_chunks_and_decode_in_one_launch(oracle_mod, Hq, Hkv):
     _mixed(oracle_mod, [1000, 7000, 0, 300, 50], [500, 1, 300, 0, 1], Hq, Hkv, 128, 256, 90)
 
 
-@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8, 12])
 @pytest.mark.parametrize("D", [64, 128])
 def test_decode_tokens_of_a_packed_batch(oracle_mod, G, D):
     """Length-1 sequences of a chunk batch at positions around the buffer
     edges (first token, just below the window, the wrap, far past it): with
-    group sizes 1 to 8 they are decoded by the decode kernel, which
+    every group size they are decoded by the decode kernel, which
     takes the token's own key and value from the packed rows (its slot still
     holds position p - W, or nothing, until the write after the attention);
     two chunks and an empty sequence share the launch."""
