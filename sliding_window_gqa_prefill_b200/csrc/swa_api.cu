@@ -133,10 +133,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Chunk attention units (all about the same cost) fill whole waves of CTAs
 // except the last; when that wave is at most half full, its pair units are
 // split into two single-head units each, which fit in it and take about three
-// quarters of a pair unit's time.  Returns the first split pair unit and
-// raises units by the number split.
+// quarters of a pair unit's time (all of them when the whole launch is at
+// most half a wave).  Returns the first split pair unit and raises units by
+// the number split.
 int split_units(int &units, int G, int sms) {
-    if (G % 2 != 0 || units <= sms || units > 0x7fffffff - sms) return units;
+    if (G % 2 != 0 || units > 0x7fffffff - sms) return units;
+    if (2 * units <= sms) {           // a launch of at most half a wave: split every unit
+        units *= 2;
+        return 0;
+    }
+    if (units <= sms) return units;
     const int rem = units % sms;
     if (rem == 0 || 2 * rem > sms) return units;
     const int from = units - rem;
@@ -406,7 +412,13 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.npairs = (G + 1) / 2;
     p.nqb = (int)nqb;
     p.num_units = (int)units;
-    p.split_from = cu_seqlens ? 0x7fffffff : (int)units;   // the lightest blocks come last: no split
+    // the lightest blocks come last, so a full launch is not split; one of at
+    // most half a wave runs as single-head units
+    p.split_from = cu_seqlens ? 0x7fffffff : (int)units;
+    if (!cu_seqlens && G % 2 == 0 && 2 * units <= dev->sms) {
+        p.split_from = 0;
+        p.num_units = (int)units * 2;
+    }
     p.scale_log2 = scale * kLog2e;
     p.chunk_mode = 0;
     p.start_pos = nullptr;
