@@ -397,6 +397,12 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             prefetch_tensormap(&tm_vs);
         }
     }
+    // a block with no unit (a packed launch whose sequences all went to the
+    // decode kernel, or fewer units than blocks) leaves before it allocates
+    // tensor memory; the test is uniform across the block
+    __syncthreads();
+    const int num_units = *unit_count;
+    if ((int)blockIdx.x >= num_units) return;
     if (warp == 2) {
         tmem_alloc(smem_addr(tmem_slot), Cfg::TMEM_COLS);
         tmem_relinquish();
@@ -405,7 +411,6 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int num_units = *unit_count;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
