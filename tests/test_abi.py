@@ -96,6 +96,29 @@ def test_workspace_size_and_status_strings(lib):
     assert lib.swa_status_string(4) == b"SWA_ERR_TIMEOUT"
 
 
+def _ws(B, Hq, Hkv, D, splits):
+    rows = B * Hq * splits
+    return ((rows * D * 4 + 255) // 256) * 256 + rows * 8
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,W,splits", [
+    (64, 32, 8, 4096, 4),      # full batch: splits of 1024 keys
+    (8, 32, 8, 4096, 4),       # 8 x 8 x 4 = 256 blocks already
+    (4, 32, 8, 4096, 8),       # small batches: shorter splits to reach ~256 blocks
+    (2, 32, 8, 4096, 16),
+    (1, 32, 8, 4096, 16),      # at least 256 keys per split
+    (1, 32, 8, 100, 1),        # a window shorter than one split
+    (3, 8, 2, 20000, 40),      # 512-key splits
+    (1, 32, 2, 4096, 16),      # group of 16: two groups of 8 per K/V head, 4 groups in all
+    (2, 22, 2, 4096, 6),       # group of 11 (prime): 11 groups of one head per K/V head (704-key splits)
+])
+def test_decode_split_policy_through_the_workspace_size(lib, B, Hq, Hkv, W, splits):
+    """The split length (1024 keys, shorter down to 256 when B times the
+    groups of the grid give under ~256 blocks) and the grouping of more than 8
+    heads per K/V head both show in the workspace size, a host-only call."""
+    assert lib.swa_decode_workspace_size(B, Hq, Hkv, 128, W) == _ws(B, Hq, Hkv, 128, splits)
+
+
 def test_every_declared_operation_has_a_python_binding():
     """Each symbol of include/swa.h is reachable from Python: a wrapper of the
     same name, the rope_theta argument of the base wrapper for the *_rope
