@@ -1,6 +1,7 @@
-"""Calls on several CUDA streams at once, as a serving process issues them:
-every kernel is deterministic, so work that overlaps on the GPU must give the
-same bits as the same calls run one after another.
+"""Determinism, and calls on several CUDA streams at once, as a serving
+process issues them: every kernel is deterministic, so repeated calls and
+work that overlaps on the GPU must give the same bits as the same calls run
+one after another.
 
 Two independent sequence sets, each with its own buffers and workspace:
 set A pre-fills in chunks and decodes on stream 1, set B takes a mixed packed
@@ -116,3 +117,27 @@ def test_overlapping_streams_give_the_sequential_bits():
         b2["vc"].copy_(vc_b0)
         torch.cuda.synchronize()
     assert swa.swa_get_device_status() == swa.SWA_OK
+
+
+def test_repeated_calls_are_bit_identical():
+    """Every entry point is deterministic: the same inputs give the same bits
+    on every call (the persistent prefill's schedule is static, the split
+    merge has a fixed order), so results reproduce exactly."""
+    B, N, Hq, Hkv, D, W = 2, 2000, 32, 8, 128, 1024
+    q, k, v = (wl.random_bf16((B, N, h, D), 7300 + i).cuda() for i, h in enumerate((Hq, Hkv, Hkv)))
+    first = swa.swa_prefill(q, k, v, W, 0.088)
+    kc = wl.random_bf16((B, W, Hkv, D), 7310).cuda()
+    vc = wl.random_bf16((B, W, Hkv, D), 7311).cuda()
+    pos = torch.tensor([5000, 900], dtype=torch.int32, device="cuda")
+    dec0 = swa.swa_decode(q[:, 0].contiguous(), kc, vc, pos, 0.088)
+    kc2, vc2 = kc.clone(), vc.clone()
+    st = torch.tensor([3000, 10], dtype=torch.int32, device="cuda")
+    ch0 = swa.swa_prefill_chunk(q[:, :W].contiguous(), k[:, :W].contiguous(), v[:, :W].contiguous(), kc2, vc2, st,
+                                W, 0.088)
+    for _ in range(3):
+        assert torch.equal(swa.swa_prefill(q, k, v, W, 0.088), first)
+        assert torch.equal(swa.swa_decode(q[:, 0].contiguous(), kc, vc, pos, 0.088), dec0)
+        kc3, vc3 = kc.clone(), vc.clone()
+        ch = swa.swa_prefill_chunk(q[:, :W].contiguous(), k[:, :W].contiguous(), v[:, :W].contiguous(), kc3, vc3,
+                                   st, W, 0.088)
+        assert torch.equal(ch, ch0) and torch.equal(kc3, kc2) and torch.equal(vc3, vc2)
