@@ -71,7 +71,9 @@ def build(force: bool = False, verbose: bool = False, debug: bool = False) -> st
 
 _lock = threading.Lock()
 _libs = {}
-_use_debug = False
+# SWA_BOUNDS_CHECK=1 in the environment makes every call of the process use
+# the index-checked library (as inside bounds_checked())
+_use_debug = os.environ.get("SWA_BOUNDS_CHECK", "") == "1"
 
 
 @contextlib.contextmanager
