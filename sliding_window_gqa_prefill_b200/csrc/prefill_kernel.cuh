@@ -64,6 +64,11 @@ struct PrefillParams {
     // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
     // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
     const int32_t *cu_seqlens;
+    // 1 (one query head per KV head, fixed-length): the two head slots of a
+    // unit are two consecutive 128-row query blocks of the same head, which
+    // share the key tiles of their bands, instead of two heads; nqb then
+    // counts those 256-row pairs
+    int qpair;
     // variable-length chunk batch: 1 leaves sequences of one row to the
     // decode kernel (no work units for them)
     int skip_len1;
@@ -186,16 +191,22 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
         P.tb = P.b;
         P.orow0 = (size_t)P.b * p.Nq;
     }
-    P.q0 = P.qb * BM;
-    P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
-    P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
+    const int span = p.qpair ? 2 * BM : BM;          // query rows of the unit
+    P.q0 = P.qb * span;
+    if (p.qpair) {
+        P.act1 = P.q0 + BM < P.nq;                   // the second block exists
+        P.h0 = P.g;
+    } else {
+        P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
+        P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
+    }
     P.nc1 = P.nc2 = 0;
     P.c1 = P.c2 = 0;
     if (!p.chunk_mode) {
         P.s0 = 0;
         P.qs = 0;
         const int lo = max(0, P.q0 - p.W + 1);
-        const int hi = min(P.nq - 1, P.q0 + BM - 1);
+        const int hi = min(P.nq - 1, P.q0 + span - 1);
         P.m0 = lo / BN;
         P.nm = hi / BN - P.m0 + 1;
         // sink positions below the band live in the first ceil(S/128) tiles
@@ -207,7 +218,7 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
             P.s0 = 0;
         }
         // sink positions j <= i - W exist for some row i of the block
-        P.sink_tile = (p.sink_buf > 0 && (long long)P.s0 + P.q0 + BM - 1 >= p.W) ? (p.sink_buf + BN - 1) / BN : 0;
+        P.sink_tile = (p.sink_buf > 0 && (long long)P.s0 + P.q0 + span - 1 >= p.W) ? (p.sink_buf + BN - 1) / BN : 0;
         P.qs = P.s0 % p.W;
         // oldest age any row of the block still needs: age < W - q0, age <= s0
         const int A = min(p.W - P.q0 - 1, P.s0);
@@ -230,7 +241,7 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
             }
         }
         const int lo = max(0, P.q0 - p.W + 1);          // chunks longer than W
-        const int hi = min(P.nq - 1, P.q0 + BM - 1);
+        const int hi = min(P.nq - 1, P.q0 + span - 1);
         P.m0 = lo / BN;
         P.nm = hi / BN - P.m0 + 1;
     }
@@ -256,6 +267,7 @@ struct TileRef {
 
 __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPlan &P, int j) {
     constexpr int BM = 128, BN = 128;
+    const int span = p.qpair ? 2 * BM : BM;          // query rows of the unit
     TileRef t;
     if (j < P.sink_tile) {                  // only the sink positions of this tile count
         t.cache = p.chunk_mode ? 2 : 0;
@@ -269,7 +281,7 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPl
         const int tile = (j < P.nc1) ? (P.c1 + j) : (P.c2 + (j - P.nc1));
         const int k0 = tile * BN;
         t.row0 = k0;
-        const int t_last = min(P.q0 + BM - 1, P.nq - 1);
+        const int t_last = min(P.q0 + span - 1, P.nq - 1);
         const bool has_qs = (k0 <= P.qs) && (P.qs < k0 + BN);
         const int max_age = (k0 + BN - 1 < P.qs) ? (P.qs - k0) : (p.W - (k0 - P.qs));
         const bool clean = !has_qs && (k0 + BN <= p.W) && (max_age < p.W - t_last) &&
@@ -279,7 +291,7 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPl
         t.cache = 0;
         const int k0 = (P.m0 + (j - P.nc1 - P.nc2)) * BN;
         t.row0 = k0;
-        const bool clean = (k0 + BN - 1 <= P.q0) && (k0 > P.q0 + BM - 1 - p.W) && (k0 + BN <= P.nq);
+        const bool clean = (k0 + BN - 1 <= P.q0) && (k0 > P.q0 + span - 1 - p.W) && (k0 + BN <= P.nq);
         t.masked = !clean;
     }
     return t;
@@ -424,12 +436,14 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int nact = 1 + P.act1;
                 if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
                 mbar_arrive_expect_tx(bar_q_full, nact * TB);
-                const int qrow = checked_coord(P.row0 + P.q0, p.Nq);
+                const int qrow = P.row0 + P.q0;
                 const int qb = checked_coord(P.tb, p.cu_seqlens ? 1 : p.B);
                 for (int t = 0; t < nact; ++t) {
-                    const int h = checked_coord(P.h0 + t, p.Hq);
+                    // the pair's second head, or with qpair its second query block
+                    const int h = checked_coord(p.qpair ? P.h0 : P.h0 + t, p.Hq);
+                    const int qr = checked_coord(qrow + (p.qpair ? t * 128 : 0), p.Nq);
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, qrow, qb);
+                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, qr, qb);
                 }
                 ++q_cnt;
                 for (int j = 0; j < P.n; ++j) {
@@ -607,7 +621,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++qc) {
             const UnitPlan P = plan_unit(p, u, pre);
             if (t == 1 && !P.act1) continue;
-            const int i_rel = P.q0 + row;                  // query row in the q tensor
+            const int i_rel = P.q0 + (p.qpair ? t * 128 : 0) + row;   // query row in the q tensor
             if (p.rope) {
                 // rotary embedding of this thread's Q row, in shared memory, at
                 // position s0 + i_rel; then make it visible to the tensor core
@@ -759,7 +773,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             ++oc;
             tc_fence_after();
-            const int h = P.h0 + t;
+            const int h = p.qpair ? P.h0 : P.h0 + t;
             bool valid_row = i_rel < P.nq;
             if (kBoundsCheck && valid_row)
                 valid_row = in_bounds((long long)P.orow0 + i_rel, p.cu_seqlens ? p.Nq : (long long)p.B * p.Nq) &&

@@ -130,6 +130,14 @@ bool bad_scale(float s) { return !(std::isfinite(s) && s > 0.f); }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// One query head per KV head (G = 1) leaves the second head slot of every
+// unit empty; with a fixed-length batch of at least two waves of units, a
+// unit takes two consecutive 128-row query blocks of one head instead (they
+// share most key tiles), which keeps both softmax warpgroups busy.
+bool use_qpair(int G, bool varlen, long long units, int sms) {
+    return G == 1 && !varlen && units >= 2LL * sms;
+}
+
 // Chunk attention units (all about the same cost) fill whole waves of CTAs
 // except the last; when that wave is at most half full, its pair units are
 // split into two single-head units each, which fit in it and take about three
@@ -412,9 +420,14 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.npairs = (G + 1) / 2;
     p.nqb = (int)nqb;
     p.num_units = (int)units;
+    if (use_qpair(G, cu_seqlens != nullptr, units, dev->sms)) {
+        p.qpair = 1;
+        p.nqb = (int)((nqb + 1) / 2);
+        p.num_units = B * Hkv * p.nqb;
+    }
     // the lightest blocks come last, so a full launch is not split; one of at
     // most half a wave runs as single-head units
-    p.split_from = cu_seqlens ? 0x7fffffff : (int)units;
+    p.split_from = cu_seqlens ? 0x7fffffff : p.num_units;
     if (!cu_seqlens && G % 2 == 0 && 2 * units <= dev->sms) {
         p.split_from = 0;
         p.num_units = (int)units * 2;
@@ -480,6 +493,11 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     p.npairs = (G + 1) / 2;
     p.nqb = (int)nqb;
     p.num_units = (int)units;
+    if (use_qpair(G, cu_seqlens != nullptr, units, dev->sms)) {
+        p.qpair = 1;
+        p.nqb = (int)((nqb + 1) / 2);
+        p.num_units = B * Hkv * p.nqb;
+    }
     p.split_from = cu_seqlens ? 0x7fffffff : split_units(p.num_units, G, dev->sms);
     p.scale_log2 = scale * kLog2e;
     p.chunk_mode = 1;
