@@ -64,10 +64,10 @@ struct PrefillParams {
     // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
     // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
     const int32_t *cu_seqlens;
-    // 1 (one query head per KV head, fixed-length): the two head slots of a
-    // unit are two consecutive 128-row query blocks of the same head, which
-    // share the key tiles of their bands, instead of two heads; nqb then
-    // counts those 256-row pairs
+    // 1 (odd group of heads, fixed-length): the two head slots of
+    // a unit are two consecutive 128-row query blocks of one head, which share
+    // the key tiles of their bands, instead of two heads of the group; npairs
+    // is then G (one head per unit) and nqb counts the 256-row pairs
     int qpair;
     // variable-length chunk batch: 1 leaves sequences of one row to the
     // decode kernel (no work units for them)
@@ -100,8 +100,9 @@ struct PrefillCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST],
-    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain, p_half[2], q_rot[2]
-    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2 + 2;
+    // v_empty[VST], s_full[2], p_full[2], o_full[2], drain, p_half[2], q_rot[2],
+    // q1_full (q_full covers Q tile 0, q1_full tile 1)
+    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2 + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base, abort flag, unit count
     static constexpr int OFF_PRE = OFF_MISC + 16;           // varlen: query-block prefix sums
     static constexpr int SMEM_BYTES = OFF_PRE + (kMaxVarlenSeqs + 1) * 4;
@@ -195,7 +196,7 @@ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, con
     P.q0 = P.qb * span;
     if (p.qpair) {
         P.act1 = P.q0 + BM < P.nq;                   // the second block exists
-        P.h0 = P.g;
+        P.h0 = P.g * p.G + P.pair;                   // one head per unit (npairs = G)
     } else {
         P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
         P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
@@ -346,6 +347,10 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t bar_drain = bar_o_full + 16;
     const uint32_t bar_p_half = bar_drain + 8;                // + 8*t
     const uint32_t bar_q_rot = bar_p_half + 16;               // + 8*t (RoPE on Q done)
+    // Q tile 1 lands on a barrier of its own: it is loaded only in units whose
+    // second head (or query block) exists, and each consumer counts the
+    // phases of the barriers it waits on over exactly those units
+    const uint32_t bar_q1_full = bar_q_rot + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::OFF_MISC + 4);
     int *unit_count = reinterpret_cast<int *>(smem + Cfg::OFF_MISC + 8);
@@ -376,6 +381,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(bar_p_half + 8, 4);
         mbar_init(bar_q_rot, 4);
         mbar_init(bar_q_rot + 8, 4);
+        mbar_init(bar_q1_full, 1);
         *abort_flag = 0;
         mbar_init_fence();
         if (p.cu_seqlens) {
@@ -429,23 +435,26 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) {
             uint32_t kc = 0, vc = 0, uc = 0;          // tiles / units issued
             uint32_t k_cnt[KST] = {}, v_cnt[VST] = {};
-            uint32_t q_cnt = 0;
+            uint32_t q_cnt = 0, q1_cnt = 0;
             bool ok = true;
             for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++uc) {
                 const UnitPlan P = plan_unit(p, u, pre);
                 const int nact = 1 + P.act1;
                 if (!mbar_wait_bounded(bar_q_empty, (uc & 1) ^ 1, abort_flag, limit)) { ok = false; break; }
-                mbar_arrive_expect_tx(bar_q_full, nact * TB);
+                mbar_arrive_expect_tx(bar_q_full, TB);
+                if (P.act1) mbar_arrive_expect_tx(bar_q1_full, TB);
                 const int qrow = P.row0 + P.q0;
                 const int qb = checked_coord(P.tb, p.cu_seqlens ? 1 : p.B);
                 for (int t = 0; t < nact; ++t) {
                     // the pair's second head, or with qpair its second query block
                     const int h = checked_coord(p.qpair ? P.h0 : P.h0 + t, p.Hq);
                     const int qr = checked_coord(qrow + (p.qpair ? t * 128 : 0), p.Nq);
+                    const uint32_t qbar = t ? bar_q1_full : bar_q_full;
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, bar_q_full, r * 64, h, qr, qb);
+                        tma_load_4d(sQ + t * TB + r * RB, &tm_q, qbar, r * 64, h, qr, qb);
                 }
                 ++q_cnt;
+                q1_cnt += P.act1;
                 for (int j = 0; j < P.n; ++j) {
                     const TileRef T = tile_ref(p, P, j);
                     const CUtensorMap *mk = T.cache == 2 ? &tm_ks : T.cache ? &tm_kc : &tm_k;
@@ -476,6 +485,7 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (!ok) {
                 // let every copy this thread started land before the block exits
                 if (q_cnt) mbar_drain_bounded(bar_q_full, (q_cnt - 1) & 1, kDrainLimitNs);
+                if (q1_cnt) mbar_drain_bounded(bar_q1_full, (q1_cnt - 1) & 1, kDrainLimitNs);
                 for (int s = 0; s < KST; ++s)
                     if (k_cnt[s]) mbar_drain_bounded(bar_k_full + 8 * s, (k_cnt[s] - 1) & 1, kDrainLimitNs);
                 for (int s = 0; s < VST; ++s)
@@ -495,24 +505,27 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t vdesc_lo = smem_desc_lo(sV, RB);
             uint32_t kc = 0, vc = 0, uc = 0;
             uint32_t pc[2] = {0, 0};
-            uint32_t qr1 = 0;                      // units with a second query head
+            uint32_t qr1 = 0;                      // units with a second query tile
             bool ok = true;
             for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++uc) {
                 const UnitPlan P = plan_unit(p, u, pre);
                 const int n = P.n;
                 if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_full, uc & 1, abort_flag, limit)) { ok = false; break; }
+                // Q tile 1 is absent in some units (odd group size, ragged last
+                // query-block pair): its barriers complete once per unit where it
+                // is present
+                if (P.act1 && !mbar_wait_bounded<Cfg::kMmaSpin>(bar_q1_full, qr1 & 1, abort_flag, limit)) {
+                    ok = false;
+                    break;
+                }
                 if (p.rope) {       // the softmax warpgroups rotate Q in place first
                     if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_rot, uc & 1, abort_flag, limit)) { ok = false; break; }
-                    // head 1 of a pair is absent in some units (odd group size): its
-                    // barrier completes once per unit where it is present
-                    if (P.act1) {
-                        if (!mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_rot + 8, qr1 & 1, abort_flag, limit)) {
-                            ok = false;
-                            break;
-                        }
-                        ++qr1;
+                    if (P.act1 && !mbar_wait_bounded<Cfg::kMmaSpin>(bar_q_rot + 8, qr1 & 1, abort_flag, limit)) {
+                        ok = false;
+                        break;
                     }
                 }
+                qr1 += P.act1;
                 // S_t = Q_t K^T for key tile j, into tensor-memory columns [t*128, t*128+128).
                 // Descriptors step along K by adding to their low word only.
                 auto issue_s = [&](int t, uint32_t kslot) {
@@ -618,14 +631,17 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float sl2 = p.scale_log2;
         uint32_t sc = 0, oc = 0, qc = 0;
         bool ok = true;
-        for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k, ++qc) {
+        for (int k = 0, u; (u = unit_of(k, blockIdx.x, gridDim.x)) < num_units && ok; ++k) {
             const UnitPlan P = plan_unit(p, u, pre);
             if (t == 1 && !P.act1) continue;
             const int i_rel = P.q0 + (p.qpair ? t * 128 : 0) + row;   // query row in the q tensor
+            // phase of this warpgroup's Q barrier: it counts only the units where
+            // the tile is loaded, like the producer's arming of it
+            const uint32_t qph = qc++ & 1;
             if (p.rope) {
                 // rotary embedding of this thread's Q row, in shared memory, at
                 // position s0 + i_rel; then make it visible to the tensor core
-                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_q_full, qc & 1, abort_flag, limit))) {
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(t ? bar_q1_full : bar_q_full, qph, abort_flag, limit))) {
                     ok = false;
                     break;
                 }

@@ -130,12 +130,15 @@ bool bad_scale(float s) { return !(std::isfinite(s) && s > 0.f); }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// One query head per KV head (G = 1) leaves the second head slot of every
-// unit empty; with a fixed-length batch of at least two waves of units, a
-// unit takes two consecutive 128-row query blocks of one head instead (they
-// share most key tiles), which keeps both softmax warpgroups busy.
+// An odd group leaves the second head slot of its last pair unit empty (all
+// of them for G = 1); with a fixed-length batch of at least two waves of
+// units, a unit takes two consecutive 128-row query blocks of one head
+// instead (they share most key tiles), which keeps both softmax warpgroups
+// busy (B=2, N=16K, W=4K: G=3 867 -> 1000, G=5 866 -> 995, G=7 854 -> 957
+// TFLOP/s).  Even groups keep the pairs of heads, which also share each key
+// tile between the two heads.
 bool use_qpair(int G, bool varlen, long long units, int sms) {
-    return G == 1 && !varlen && units >= 2LL * sms;
+    return G % 2 == 1 && !varlen && units >= 2LL * sms;
 }
 
 // Chunk attention units (all about the same cost) fill whole waves of CTAs
@@ -422,8 +425,9 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     p.num_units = (int)units;
     if (use_qpair(G, cu_seqlens != nullptr, units, dev->sms)) {
         p.qpair = 1;
+        p.npairs = G;
         p.nqb = (int)((nqb + 1) / 2);
-        p.num_units = B * Hkv * p.nqb;
+        p.num_units = B * Hkv * G * p.nqb;
     }
     // the lightest blocks come last, so a full launch is not split; one of at
     // most half a wave runs as single-head units
@@ -495,8 +499,9 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     p.num_units = (int)units;
     if (use_qpair(G, cu_seqlens != nullptr, units, dev->sms)) {
         p.qpair = 1;
+        p.npairs = G;
         p.nqb = (int)((nqb + 1) / 2);
-        p.num_units = B * Hkv * p.nqb;
+        p.num_units = B * Hkv * G * p.nqb;
     }
     p.split_from = cu_seqlens ? 0x7fffffff : split_units(p.num_units, G, dev->sms);
     p.scale_log2 = scale * kLog2e;

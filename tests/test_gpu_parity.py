@@ -355,22 +355,26 @@ def test_decode_bindings_check_the_key_cache_shape():
 
 # ------------------------------------------------------------------ one query head per KV head
 
-@pytest.mark.parametrize("B,N,H,D,W", [
-    (1, 1900, 32, 128, 500),     # 15 query blocks: the last pair holds one block
-    (2, 1280, 16, 64, 300),      # D=64, an even number of blocks
-    (1, 2048, 32, 128, 3000),    # window wider than the sequence
+@pytest.mark.parametrize("B,N,Hq,H,D,W", [
+    (1, 1900, 32, 32, 128, 500),     # one head per KV head; 15 query blocks: the last pair holds one
+    (2, 1280, 16, 16, 64, 300),      # D=64, an even number of blocks
+    (1, 2048, 32, 32, 128, 3000),    # window wider than the sequence
+    (1, 2560, 24, 8, 128, 600),      # groups of 3
+    (1, 1700, 40, 8, 64, 450),       # groups of 5, ragged last pair, D=64
+    (1, 1300, 56, 8, 128, 700),      # groups of 7
 ])
-def test_mha_units_of_two_query_blocks(oracle_mod, B, N, H, D, W):
-    """Hq == Hkv (one query head per KV head) with at least two waves of units:
-    a unit takes two consecutive 128-row query blocks of one head (key tiles
-    of both bands, masked per row), plain, with RoPE on q and with sinks."""
+def test_odd_groups_in_units_of_two_query_blocks(oracle_mod, B, N, Hq, H, D, W):
+    """Odd groups (1, 3, 5, 7 query heads per KV head) with at least two waves
+    of units: a unit takes two consecutive 128-row query blocks of one head (key
+    tiles of both bands, masked per row), plain, with RoPE on q and with
+    sinks."""
     seed = 8000 + N + H
-    q = wl.random_bf16((B, N, H, D), seed)
+    q = wl.random_bf16((B, N, Hq, D), seed)
     k = wl.random_bf16((B, N, H, D), seed + 1)
     v = wl.random_bf16((B, N, H, D), seed + 2)
     scale = 1.0 / math.sqrt(D)
     out = run_prefill(q, k, v, W, scale)
-    assert_close(out, oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale), f"MHA B{B} N{N} D{D} W{W}")
+    assert_close(out, oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale), f"G={Hq // H} B{B} N{N} D{D} W{W}")
     outr = swa.swa_prefill(q.cuda(), k.cuda(), v.cuda(), W, scale, rope_theta=10000.0)
     qr = oracle_mod.rope(f64(q), np.zeros(B, np.int32), 10000.0)
     assert_close(outr.cpu(), oracle_mod.swa_prefill(qr, f64(k), f64(v), W, scale), f"MHA RoPE N{N}")
@@ -378,13 +382,14 @@ def test_mha_units_of_two_query_blocks(oracle_mod, B, N, H, D, W):
     assert_close(outs.cpu(), oracle_mod.swa_prefill_sinks(f64(q), f64(k), f64(v), W, 4, scale), f"MHA sinks N{N}")
 
 
-def test_mha_chunked_units_of_two_query_blocks(oracle_mod):
-    """Chunked prefill with one query head per KV head (10 query blocks of 32
-    heads per chunk: 320 units, so pairs of blocks): every row against one-shot
-    SWA, the buffer bit for bit."""
-    B, N, C, H, D, W = 1, 2560, 1280, 32, 128, 1280
-    q, k, v, scale, out, kc, vc = _chunked_case(oracle_mod, B, N, C, H, H, D, W, seed=8100)
-    assert_close(out, oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale), "MHA chunked")
+@pytest.mark.parametrize("Hq,H", [(32, 32), (24, 8)])
+def test_odd_groups_chunked_in_units_of_two_query_blocks(oracle_mod, Hq, H):
+    """Chunked prefill with groups of 1 and 3 (10 query blocks per chunk: 320
+    head-pair units, so pairs of blocks): every row against one-shot SWA, the
+    buffer bit for bit."""
+    B, N, C, D, W = 1, 2560, 1280, 128, 1280
+    q, k, v, scale, out, kc, vc = _chunked_case(oracle_mod, B, N, C, Hq, H, D, W, seed=8100 + Hq)
+    assert_close(out, oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale), f"G={Hq // H} chunked")
     for s in range(W):
         p = s + ((N - 1 - s) // W) * W
         assert torch.equal(kc[:, s], k[:, p]) and torch.equal(vc[:, s], v[:, p]), (s, p)

@@ -91,9 +91,33 @@ def test_prefill_rope_fused_q(oracle_mod, B, N, Hq, Hkv, D, W):
     close(out, ref, "prefill rope")
 
 
+@pytest.mark.parametrize("B,N,Hq,Hkv,D,W", [
+    (1, 2304, 24, 8, 128, 600),      # groups of 3 in head pairs: 288 units, 70 blocks take a one-head unit first
+    (1, 1300, 56, 8, 128, 700),      # groups of 7 in query-block pairs: 56 blocks start on the one-block pair
+    (1, 1280, 24, 8, 64, 300),       # groups of 3, 160 units: 6 blocks take a one-head unit, then a pair (D=64)
+])
+def test_prefill_rope_second_q_tile_absent_then_present(oracle_mod, B, N, Hq, Hkv, D, W):
+    """Persistent blocks whose unit has no second Q tile (the last head of an
+    odd group, or a last query-block pair with one block) and whose next unit
+    has one: the warpgroup that rotates tile 1 waits for that tile's own load
+    and rotates it exactly once."""
+    seed = 6900 + N + Hq
+    q = wl.random_bf16((B, N, Hq, D), seed)
+    k = wl.random_bf16((B, N, Hkv, D), seed + 1)
+    v = wl.random_bf16((B, N, Hkv, D), seed + 2)
+    scale = 1 / math.sqrt(D)
+    zero = np.zeros(B, np.int32)
+    for _ in range(2):
+        out = swa.swa_prefill(q.cuda(), k.cuda(), v.cuda(), W, scale, rope_theta=THETA)
+        torch.cuda.synchronize()
+        ref = oracle_mod.swa_prefill(oracle_mod.rope(f64(q), zero, THETA), f64(k), f64(v), W, scale)
+        close(out, ref, f"prefill rope G={Hq // Hkv} N{N}")
+
+
 @pytest.mark.parametrize("B,N,C,Hq,Hkv,D,W", [
     (2, 520, 200, 8, 2, 128, 256),
     (1, 2560, 1280, 32, 4, 64, 1280),    # 160 units: the last wave split into single-head units, G=8, D=64
+    (1, 2560, 1280, 24, 8, 128, 1280),   # groups of 3: blocks that take a one-head unit, then a pair
 ])
 def test_chunked_rope_then_decode_rope_continue_the_sequence(oracle_mod, B, N, C, Hq, Hkv, D, W):
     """Chunks with q rotated at load and keys rotated before the chunk call,
