@@ -382,12 +382,12 @@ def test_odd_groups_in_units_of_two_query_blocks(oracle_mod, B, N, Hq, H, D, W):
     assert_close(outs.cpu(), oracle_mod.swa_prefill_sinks(f64(q), f64(k), f64(v), W, 4, scale), f"MHA sinks N{N}")
 
 
-@pytest.mark.parametrize("Hq,H", [(32, 32), (24, 8)])
-def test_odd_groups_chunked_in_units_of_two_query_blocks(oracle_mod, Hq, H):
+@pytest.mark.parametrize("B,Hq,H", [(1, 32, 32), (2, 24, 8)])
+def test_odd_groups_chunked_in_units_of_two_query_blocks(oracle_mod, B, Hq, H):
     """Chunked prefill with groups of 1 and 3 (10 query blocks per chunk: 320
-    head-pair units, so pairs of blocks): every row against one-shot SWA, the
-    buffer bit for bit."""
-    B, N, C, D, W = 1, 2560, 1280, 128, 1280
+    head-pair units either way, so pairs of blocks): every row against
+    one-shot SWA, the buffer bit for bit."""
+    N, C, D, W = 2560, 1280, 128, 1280
     q, k, v, scale, out, kc, vc = _chunked_case(oracle_mod, B, N, C, Hq, H, D, W, seed=8100 + Hq)
     assert_close(out, oracle_mod.swa_prefill(f64(q), f64(k), f64(v), W, scale), f"G={Hq // H} chunked")
     for s in range(W):
