@@ -121,6 +121,7 @@ struct PrefillCfg {
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, 1);
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(SMEM_ALLOC <= 232448, "dynamic shared memory of one block (227 KB)");
 };
 
 // Which query rows and key tiles one work unit covers.
