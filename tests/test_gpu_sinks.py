@@ -87,6 +87,8 @@ def test_streaming_decode_with_sinks(oracle_mod, W, S, D):
     (1, 1000, 300, 6, 2, 128, 384, 130),  # two sink tiles, odd group
     (2, 2560, 1280, 16, 4, 128, 1536, 4),  # last wave split into single-head units, with a sink tile
     (1, 600, 200, 16, 1, 64, 256, 4),      # group of 16: decode as two groups of 8 on the same K/V head
+    (2, 2600, 1280, 24, 8, 128, 1280, 4),  # groups of 3, 320 units: pairs of query blocks; a 40-row last chunk
+    (1, 2560, 1280, 32, 32, 64, 1280, 130),  # one head per KV head in pairs of query blocks, two sink tiles
 ])
 def test_chunked_prefill_with_sinks(oracle_mod, B, N, C, Hq, Hkv, D, W, S):
     """Chunks through the rolling buffer with the sink buffer: the outputs equal
