@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
     ap.add_argument("--log", default=None,
                     help="also append the result, and one row per measured part, as JSON lines to this file")
-    ap.add_argument("--ncu-case", choices=["prefill", "prefill_b2", "chunk", "decode", "mixed"], default=None,
+    ap.add_argument("--ncu-case", choices=["prefill", "prefill_b2", "chunk", "decode", "decode_w8k", "mixed"], default=None,
                     help="run a reduced case of one kernel three times for an ncu capture (no timing)")
     return ap.parse_args(argv)
 
@@ -180,6 +180,25 @@ def weak_scaling_rate(units_per_rank: float, world: int, max_seconds: float) -> 
     """Whole-job throughput: every rank processes the same units; the job
     takes as long as its slowest rank."""
     return units_per_rank * world / max_seconds
+
+
+def decode_splits(swa, B: int, Hq: int, Hkv: int, D: int, W: int) -> int:
+    """Splits per window of a swa_decode call, read back from its workspace
+    size (rows = B * Hq * splits of D floats, 256-byte padded, then one (m, l)
+    pair per row)."""
+    n = swa.swa_decode_workspace_size(B, Hq, Hkv, D, W)
+    for splits in range(1, 4097):
+        rows = B * Hq * splits
+        if (rows * D * 4 + 255) // 256 * 256 + rows * 8 == n:
+            return splits
+    raise RuntimeError("decode workspace size matches no split count")
+
+
+def decode_kernels_per_call(splits: int) -> int:
+    """Kernels one swa_decode call (no sinks) launches: the split-KV kernel,
+    plus the split merge unless the window is one split or exactly four
+    (merged on chip by the four blocks of a cluster)."""
+    return 1 if splits in (1, 4) else 2
 
 
 def barrier(world: int):
@@ -380,7 +399,7 @@ def run_native(args):
     dec_tok_s = weak_scaling_rate(dw.B * dw.steps * args.steps, world, de_total * 1e-3)
     dec_gbs = (kv_bytes + other_bytes) / ((de_total / args.steps) * 1e-3) / 1e9
     dec_kv_gbs = kv_bytes / ((de_total / args.steps) * 1e-3) / 1e9
-    # roofline of the dominant launch (decode: split-KV kernel + merge), bytes
+    # roofline of the dominant launch (decode: split-KV kernel and its merge), bytes
     # it must move per call (K/V rows in the window, q in, out back) over the
     # event-timed duration of the calls
     dec_call_ms = max_over_ranks(dec_call_ms, world)
@@ -443,9 +462,10 @@ def run_native(args):
     pcie["frac_of_both_at_once"] = pcie["both_ms"] / (e2e_ms / args.steps)
 
     # per step: the one-shot prefill, attention + append per chunk, and per
-    # decode step the append, the split-KV kernel and the split merge (the
-    # window of 4096 keys spans several 1024-key splits, so the merge runs)
-    launches_per_step = 1 + len(c_chunks) * 2 + dw.steps * 3
+    # decode step the append and the decode kernels (at B=64 the 4096-key
+    # window is 4 splits of 1024 keys, merged in a cluster: no merge launch)
+    dec_splits = decode_splits(swa, dw.B, dw.Hq, dw.Hkv, dw.D, dw.W)
+    launches_per_step = 1 + len(c_chunks) * 2 + dw.steps * (1 + decode_kernels_per_call(dec_splits))
 
     # ---- the widened rows, timed on their own (CUDA events, after the step)
     extras = measure_extras(swa, wl, dev, q, k, v, hp, dd, dw, max(3, args.steps // 2), world)
@@ -478,7 +498,10 @@ def run_native(args):
             "config": bench_config(hp, world),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "swa_decode (swa_decode_kernel<128,4> + swa_decode_combine_kernel<128,4>)",
+                "kernel": ("swa_decode (swa_decode_kernel<128,4>, its 4 splits merged in a cluster)"
+                           if decode_kernels_per_call(dec_splits) == 1 and dec_splits == 4 else
+                           "swa_decode (swa_decode_kernel<128,4> + swa_decode_combine_kernel<128,4>)"),
+                "splits_per_window": dec_splits,
                 "why_this_kernel": "largest share of the step's GPU time (ncu launch list and events)",
                 "achieved": dec_call_gbs,
                 "peak": peaks["hbm_gbs"],
@@ -747,7 +770,9 @@ def run_ncu_case(case: str) -> None:
     on the device), `prefill` half of it (B=1, same per-unit structure),
     `chunk` the benchmark's chunked prefill (4 x attention + append), `decode`
     a reduced decode (B=16, a quarter of the batch, positions from the same
-    distribution, still above L2), `mixed` the benchmark's mixed packed call
+    distribution, still above L2; 4 splits per window, merged in a cluster),
+    `decode_w8k` the same batch with an 8192-slot buffer (8 splits per
+    window, so the split merge kernel runs), `mixed` the benchmark's mixed packed call
     (4 chunks of 4096 and 60 decode tokens over the decode workload's 1 GB of
     buffers; its decode tokens run in the decode kernel's cluster mode).
     Prints the algorithmic bytes per launch so a capture's DRAM traffic can be
@@ -804,7 +829,7 @@ def run_ncu_case(case: str) -> None:
         print(f"ncu case mixed: decode-token launch algorithmic bytes {alg} (K/V rows in the 60 windows, "
               f"the own rows included, + q + out rows)")
     else:
-        w = dataclasses.replace(wl.DECODE_B64, B=16, steps=1)
+        w = dataclasses.replace(wl.DECODE_B64, B=16, steps=1, W=8192 if case == "decode_w8k" else wl.DECODE_B64.W)
         d = wl.decode_inputs(w)
         kc, vc, pos = d["k_cache"].cuda(), d["v_cache"].cuda(), d["pos0"].cuda()
         q = d["q"][0].cuda().contiguous()
@@ -814,8 +839,8 @@ def run_ncu_case(case: str) -> None:
             swa.swa_decode(q, kc, vc, pos, w.scale, workspace=ws)
         keys = sum(min(int(p) + 1, w.W) for p in d["pos0"])
         alg = keys * w.Hkv * w.D * 2 * 2 + q.numel() * 2 * 2
-        print(f"ncu case decode B=16 W={w.W}: algorithmic bytes per launch {alg} (K/V rows in the window "
-              f"+ q + out)")
+        print(f"ncu case {case} B=16 W={w.W}: algorithmic bytes per launch {alg} (K/V rows in the window "
+              f"+ q + out), {decode_splits(swa, w.B, w.Hq, w.Hkv, w.D, w.W)} splits per window")
     torch.cuda.synchronize()
     if swa.swa_get_device_status() != 0:
         raise SystemExit("device status not OK")

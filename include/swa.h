@@ -138,6 +138,9 @@ swa_status_t swa_cache_append(const void *k_new, const void *v_new,
  * workspace: device scratch of at least swa_decode_workspace_size() bytes,
  *   256-byte aligned, owned by the caller; its contents need no set-up and are
  *   overwritten.  Calls that share a workspace must not overlap on the GPU.
+ *   When the window takes exactly 4 splits (without sinks) the splits are
+ *   merged on chip and the workspace is left untouched; it is still checked
+ *   and must still be passed.
  */
 swa_status_t swa_decode(const void *q, const void *k_cache, const void *v_cache,
                         const int32_t *pos, void *out, int B, int Hq, int Hkv,

@@ -28,12 +28,15 @@
 //    rescale of l and o) only when a score exceeds it by more than 2^8, so
 //    most blocks take no maximum.
 //  * warps and splits are merged by log-sum-exp: in shared memory inside a
-//    block, and by swa_decode_combine_kernel across splits.
+//    block, and across splits either by swa_decode_combine_kernel or, when a
+//    window takes exactly 4 splits (W = 4096 at large batch), inside a
+//    cluster of those 4 blocks through distributed shared memory (one
+//    launch fewer per step: 146.7 vs 149.7 us per call at B=64, W=4096).
 //  * the one-token sequences of a packed chunk batch (decode steps in a
 //    mixed pre-fill call) take a third mode: the token's own K/V come from
 //    its packed row (the buffer is written after the attention), and the 4
-//    splits of a window are the blocks of one cluster, merged through
-//    distributed shared memory instead of a workspace.
+//    splits of a window are the blocks of one cluster, merged the same way,
+//    so no workspace is needed.
 #pragma once
 
 #include "device_common.cuh"
@@ -48,9 +51,8 @@ constexpr int kDecodeMinSplit = 256;
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeBlk = 16;         // keys per tensor-core block
 constexpr int kDecodeStages = 3;       // per-warp ring depth, in 16-key blocks
-// MODE 2 (length-1 sequences of a packed chunk batch, no workspace): the
-// window of one (sequence, kv head) is split over a cluster of this many
-// blocks, merged through distributed shared memory
+// MODE 2 and 3 (no workspace): the window of one (sequence, kv head) is split
+// over a cluster of this many blocks, merged through distributed shared memory
 constexpr int kDecodeClusterSplits = 4;
 
 template <int D, int G>
@@ -131,8 +133,9 @@ __device__ __forceinline__ uint32_t swz_off(int r, int ch, int row_bytes) {
 // are row cu[b] of the packed k and v, passed as ksink / vsink.  The window
 // is split over a cluster of kDecodeClusterSplits blocks (grid x), merged
 // through distributed shared memory (each block merges a quarter of the
-// outputs from all blocks' partials), so no workspace is needed.
-constexpr int kDecodeWindow = 0, kDecodeSinks = 1, kDecodePackedRows = 2;
+// outputs from all blocks' partials), so no workspace is needed.  MODE 3: the
+// window as in MODE 0, split and merged as in MODE 2.
+constexpr int kDecodeWindow = 0, kDecodeSinks = 1, kDecodePackedRows = 2, kDecodeWindowCluster = 3;
 
 template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
@@ -144,6 +147,8 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                   const __nv_bfloat16 *__restrict__ vsink, int S, const int32_t *__restrict__ cu,
                   int total, int split_len, int kv_rep) {
     constexpr bool SINKS = MODE == kDecodeSinks;
+    // the splits of a window are the blocks of one cluster (grid x)
+    constexpr bool CLUSTER = MODE == kDecodePackedRows || MODE == kDecodeWindowCluster;
     using Cfg = DecodeCfg<D, G>;
     constexpr int CH = Cfg::CH, RB = Cfg::ROW_BYTES;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -174,9 +179,9 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const int L = Lw + ns;
     constexpr int kClusterKeys = kDecodeClusterSplits * kDecodeBlk;
     const int split_keys =
-        (MODE == kDecodePackedRows) ? (L + kClusterKeys - 1) / kClusterKeys * kDecodeBlk : split_len;
-    // MODE 2: a block past the window's keys still takes part in the merge
-    if (MODE != kDecodePackedRows && split * split_keys >= L) return;
+        CLUSTER ? (L + kClusterKeys - 1) / kClusterKeys * kDecodeBlk : split_len;
+    // a cluster block past the window's keys still takes part in the merge
+    if (!CLUSTER && split * split_keys >= L) return;
     const int begin = min(split * split_keys, L);
     const int end = min(L, begin + split_keys);
     const int nsplit = (L + split_keys - 1) / split_keys;
@@ -366,7 +371,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         }
     }
     __syncthreads();
-    float *part = mg + kDecodeWarps * G * (D + 2);  // [G][D+2]: the block's merge (MODE 2)
+    float *part = mg + kDecodeWarps * G * (D + 2);  // [G][D+2]: the block's merge (cluster modes)
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D, d = idx % D;
         float m = -INFINITY;
@@ -380,7 +385,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             l += src[D + 1] * sc;
             acc += src[d] * sc;
         }
-        if (MODE == kDecodePackedRows) {
+        if (CLUSTER) {
             part[h * (D + 2) + d] = acc;
             if (d == 0) {
                 part[h * (D + 2) + D] = m;
@@ -396,7 +401,7 @@ swa_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             if (d == 0) ws_ml[slot] = make_float2(m, l);
         }
     }
-    if constexpr (MODE == kDecodePackedRows) {
+    if constexpr (CLUSTER) {
         // every block of the cluster reaches both barriers: the only returns
         // above depend on (b) alone, which the cluster shares
         cluster_sync_all();

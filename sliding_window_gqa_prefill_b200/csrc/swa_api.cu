@@ -105,6 +105,9 @@ swa_status_t device_info(DeviceInfo **out) {
                                       swa::DecodeCfg<DD, GG>::SMEM_BYTES));                  \
     SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, swa::kDecodePackedRows>, \
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                      swa::DecodeCfg<DD, GG>::SMEM_BYTES));                  \
+    SWA_CUDA_TRY(cudaFuncSetAttribute(swa::swa_decode_kernel<DD, GG, swa::kDecodeWindowCluster>, \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,           \
                                       swa::DecodeCfg<DD, GG>::SMEM_BYTES));
         SWA_SET_DECODE_ATTR(64, 1) SWA_SET_DECODE_ATTR(64, 2) SWA_SET_DECODE_ATTR(64, 3)
         SWA_SET_DECODE_ATTR(64, 4) SWA_SET_DECODE_ATTR(64, 5) SWA_SET_DECODE_ATTR(64, 6)
@@ -223,6 +226,39 @@ int decode_nsplit_max(int B, int Hkv, int L) {
     return (int)(((long long)L + split - 1) / split);
 }
 
+// Grid (kDecodeClusterSplits, Hkv, B) in clusters of kDecodeClusterSplits
+// along x: the splits of each window are merged through distributed shared
+// memory, with no workspace.  MODE kDecodeWindowCluster: the window of the
+// cache (knew / vnew / cu unused, total = B); kDecodePackedRows: the
+// one-row sequences of a packed batch.
+template <int D, int G, int MODE>
+swa_status_t launch_decode_cluster(const void *q, const void *kc, const void *vc, const int32_t *pos,
+                                   void *out, int B, int Hkv, int W, float scale,
+                                   const swa::RopeTable *rope, const void *knew, const void *vnew,
+                                   const int32_t *cu, int total, int kv_rep, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(swa::kDecodeClusterSplits, Hkv, B);
+    cfg.blockDim = dim3(swa::kDecodeWarps * 32);
+    cfg.dynamicSmemBytes = swa::DecodeCfg<D, G>::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = swa::kDecodeClusterSplits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    float2 *no_ml = nullptr;
+    float *no_o = nullptr;
+    SWA_CUDA_TRY(cudaLaunchKernelEx(&cfg, swa::swa_decode_kernel<D, G, MODE>,
+                                    static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(kc),
+                                    static_cast<const __nv_bfloat16 *>(vc), pos, static_cast<__nv_bfloat16 *>(out),
+                                    no_ml, no_o, Hkv, W, 1, scale * kLog2e, rope ? 1 : 0,
+                                    rope ? *rope : swa::RopeTable{}, static_cast<const __nv_bfloat16 *>(knew),
+                                    static_cast<const __nv_bfloat16 *>(vnew), 0, cu, total, 0, kv_rep));
+    return SWA_OK;
+}
+
 // Hkv: groups of G query heads (kv_rep groups per K/V head in memory).
 template <int D, int G>
 swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, const int32_t *pos,
@@ -235,6 +271,10 @@ swa_status_t launch_decode_dg(const void *q, const void *kc, const void *vc, con
     float *ws_o = static_cast<float *>(ws);
     float2 *ws_ml = ws ? reinterpret_cast<float2 *>(static_cast<char *>(ws) + ((o_elems * 4 + 255) & ~size_t(255)))
                        : nullptr;
+    // a window of exactly kDecodeClusterSplits splits: merged in its cluster
+    if (S == 0 && nsm == swa::kDecodeClusterSplits)
+        return launch_decode_cluster<D, G, swa::kDecodeWindowCluster>(q, kc, vc, pos, out, B, Hkv, W, scale, rope,
+                                                                      nullptr, nullptr, nullptr, B, kv_rep, s);
     dim3 grid(nsm, Hkv, B);
     auto kernel = S > 0 ? swa::swa_decode_kernel<D, G, swa::kDecodeSinks>
                         : swa::swa_decode_kernel<D, G, swa::kDecodeWindow>;
@@ -279,30 +319,8 @@ swa_status_t launch_decode_packed_dg(const void *q, const void *k, const void *v
                                      const void *vc, const int32_t *start_pos, const int32_t *cu,
                                      void *out, int B, int total, int Hkv, int W, float scale,
                                      cudaStream_t s, int kv_rep) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(swa::kDecodeClusterSplits, Hkv, B);
-    cfg.blockDim = dim3(swa::kDecodeWarps * 32);
-    cfg.dynamicSmemBytes = swa::DecodeCfg<D, G>::SMEM_BYTES;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = swa::kDecodeClusterSplits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q);
-    const __nv_bfloat16 *kcb = static_cast<const __nv_bfloat16 *>(kc);
-    const __nv_bfloat16 *vcb = static_cast<const __nv_bfloat16 *>(vc);
-    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(k);
-    const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(v);
-    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(out);
-    float2 *no_ml = nullptr;
-    float *no_o = nullptr;
-    SWA_CUDA_TRY(cudaLaunchKernelEx(&cfg, swa::swa_decode_kernel<D, G, swa::kDecodePackedRows>, qb, kcb, vcb,
-                                    start_pos, ob, no_ml, no_o, Hkv, W, 1, scale * kLog2e, 0, swa::RopeTable{},
-                                    kb, vb, 0, cu, total, 0, kv_rep));
-    return SWA_OK;
+    return launch_decode_cluster<D, G, swa::kDecodePackedRows>(q, kc, vc, start_pos, out, B, Hkv, W, scale, nullptr,
+                                                               k, v, cu, total, kv_rep, s);
 }
 
 // false when the decode kernel has no instance for this head group

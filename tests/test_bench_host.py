@@ -118,3 +118,15 @@ def test_log_rows_one_per_measured_part(tmp_path):
     assert rows[-1]["value"] == 2.1 and rows[2]["tflops"] == 2.0
     bench.write_log(str(path), res)
     assert len(path.read_text().splitlines()) == 2 * len(rows)
+
+
+def test_decode_launch_count_follows_the_split_policy():
+    """bench.py counts one decode kernel per call for windows of one or four
+    splits (merged on chip) and two otherwise; the split count is read back
+    from the workspace size."""
+    import sliding_window_gqa_prefill_b200 as swa
+    swa.build()
+    assert bench.decode_splits(swa, 64, 32, 8, 128, 4096) == 4
+    assert bench.decode_splits(swa, 2, 32, 8, 128, 4096) == 16
+    assert bench.decode_splits(swa, 1, 32, 8, 128, 100) == 1
+    assert [bench.decode_kernels_per_call(n) for n in (1, 2, 4, 8, 16)] == [1, 2, 1, 2, 2]

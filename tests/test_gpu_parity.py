@@ -248,6 +248,36 @@ def test_decode_edge_cases(oracle_mod, B, Hq, Hkv, D, W, pos0):
     _decode_case(oracle_mod, B, Hq, Hkv, D, W, pos0, steps=3, seed=B * W + D)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,D,W,pos0", [
+    (8, 32, 8, 128, 4096, [0, 1, 17, 63, 64, 4094, 4095, 9000]),  # 4 splits of 1024; short windows leave blocks empty
+    (2, 4, 2, 64, 1000, [5, 30000]),                              # 4 splits of 256 (small batch), D=64
+    (4, 96, 8, 128, 1024, [1023, 3, 5000, 700]),                  # group of 12: two groups of 6 per K/V head
+])
+def test_decode_windows_of_four_splits_merge_in_a_cluster(oracle_mod, B, Hq, Hkv, D, W, pos0):
+    """A window cut into exactly 4 splits (the W=4096 decode at large batch) is
+    merged on chip by the 4 blocks of a cluster: outputs against the oracle,
+    plain and with RoPE on q, and the caller's workspace left as it was."""
+    kc = wl.random_bf16((B, W, Hkv, D), 9100 + W)
+    vc = wl.random_bf16((B, W, Hkv, D), 9101 + W)
+    q = wl.random_bf16((B, Hq, D), 9102 + W)
+    pos = torch.tensor(pos0, dtype=torch.int32)
+    scale = 1.0 / math.sqrt(D)
+    sp = oracle_mod.slot_positions((pos + 1).numpy(), W)     # the token at pos is already in the buffer
+    need = swa.swa_decode_workspace_size(B, Hq, Hkv, D, W)
+    assert need > 0
+    ws = torch.full((need,), 0x5A, dtype=torch.uint8, device="cuda")
+    kg, vg, pg = kc.cuda(), vc.cuda(), pos.cuda()
+    out = swa.swa_decode(q.cuda(), kg, vg, pg, scale, workspace=ws)
+    outr = swa.swa_decode(q.cuda(), kg, vg, pg, scale, workspace=ws, rope_theta=10000.0)
+    torch.cuda.synchronize()
+    assert bool((ws == 0x5A).all()), "the on-chip merge leaves the workspace untouched"
+    ref = oracle_mod.swa_decode(f64(q), f64(kc), f64(vc), sp, pos.numpy(), W, scale)
+    assert_close(out.cpu(), ref, f"4-split decode B{B} W{W} G{Hq // Hkv}")
+    qr = oracle_mod.rope(f64(q)[:, None], pos.numpy(), 10000.0)[:, 0]
+    refr = oracle_mod.swa_decode(qr, f64(kc), f64(vc), sp, pos.numpy(), W, scale)
+    assert_close(outr.cpu(), refr, f"4-split decode RoPE B{B} W{W}")
+
+
 def test_prefill_then_decode_continues_the_sequence(oracle_mod):
     """Chunked prefill leaves the buffer in the state decode continues from:
     decode at position N equals row N of one-shot SWA over N+1 tokens."""
