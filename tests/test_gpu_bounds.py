@@ -125,6 +125,7 @@ def test_packed_batches():
     (4, 32, 8, 128, 4096, [0, 1, 4094, 4095]), (3, 8, 2, 128, 4096, [4096, 8191, 30000]),
     (2, 4, 4, 64, 700, [10, 2000]), (2, 16, 2, 128, 1000, [999, 5]), (2, 4, 2, 64, 300, [299, 77]),
     (2, 8, 2, 128, 8192, [8191, 20000]), (1, 4, 1, 64, 5000, [4999]),
+    (8, 32, 8, 128, 4096, [0, 1, 17, 63, 64, 4095, 4096, 9000]),   # 4 splits per window: merged in a cluster
 ])
 def test_append_and_decode(B, Hq, Hkv, D, W, pos0):
     pos = torch.tensor(pos0, dtype=torch.int32, device="cuda")
