@@ -64,7 +64,7 @@ def load_peaks():
 
 # the sources each kernel is built from (its launch code is in swa_api.cu)
 KERNEL_SOURCES = {
-    "swa_prefill_kernel<128>": ("device_common.cuh", "prefill_kernel.cuh", "swa_api.cu"),
+    "swa_prefill_kernel<128>": ("device_common.cuh", "prefill_plan.cuh", "prefill_kernel.cuh", "swa_api.cu"),
     "swa_decode_kernel<128,4>": ("device_common.cuh", "decode_kernel.cuh", "swa_api.cu"),
 }
 

@@ -34,7 +34,7 @@ LIB_PATH = os.path.join(_PKG, "libswa.so")
 DEBUG_LIB_PATH = os.path.join(_PKG, "libswa_debug.so")
 HEADER = os.path.join(_ROOT, "include", "swa.h")
 _SOURCES = [os.path.join(_PKG, "csrc", f) for f in
-            ("swa_api.cu", "device_common.cuh", "prefill_kernel.cuh", "decode_kernel.cuh")]
+            ("swa_api.cu", "device_common.cuh", "prefill_plan.cuh", "prefill_kernel.cuh", "decode_kernel.cuh")]
 
 SWA_OK, SWA_ERR_INVALID_ARG, SWA_ERR_UNSUPPORTED, SWA_ERR_CUDA, SWA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 SWA_WINDOW_EXCL_LEFT, SWA_WINDOW_INCL_LEFT = 0, 1

@@ -38,50 +38,10 @@
 //    returns).
 #pragma once
 
-#include "device_common.cuh"
+#include "prefill_plan.cuh"
 
 namespace swa {
 
-struct PrefillParams {
-    int B;            // sequences
-    int Nq;           // query rows per sequence (N, or C in chunk mode)
-    int Nk;           // rows of the main k/v tensors (== Nq)
-    int Hq, Hkv, G;   // heads, G = Hq / Hkv
-    int W;            // window (keys i-W < j <= i)
-    int npairs;       // ceil(G / 2)
-    int nqb;          // ceil(Nq / 128)
-    int num_units;    // B * Hkv * npairs * nqb, plus one per pair unit split in two
-    // pair units with index >= split_from are split into two single-head units
-    // (fills the last wave of CTAs; == the pair-unit count when nothing is split)
-    int split_from;
-    float scale_log2; // softmax scale * log2(e)
-    int chunk_mode;   // 1: keys also come from the rolling-buffer cache
-    const int32_t *start_pos;  // chunk mode: [B] first position of the chunk
-    __nv_bfloat16 *out;        // [B, Nq, Hq, D]
-    int out_v8;                // 1: out is 32-byte aligned (rows of 128 or 256 bytes): 32-byte stores
-    int rope;                  // 1: rotate each Q tile in shared memory after its load
-    RopeTable rope_freq;       // theta^(-2i/D), i < D/2
-    // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
-    // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
-    const int32_t *cu_seqlens;
-    // 1 (odd group of heads, fixed-length): the two head slots of
-    // a unit are two consecutive 128-row query blocks of one head, which share
-    // the key tiles of their bands, instead of two heads of the group; npairs
-    // is then G (one head per unit) and nqb counts the 256-row pairs
-    int qpair;
-    // variable-length chunk batch: 1 leaves sequences of one row to the
-    // decode kernel (no work units for them)
-    int skip_len1;
-    // attention sinks (one-shot prefill): positions j < sinks stay visible to
-    // every query besides its window
-    int sinks;
-    // attention sinks (chunk mode): slots 0 .. sink_buf-1 of the sink buffer
-    // hold positions 0 .. sink_buf-1; those outside a query's window are
-    // visible to it (0: no sinks)
-    int sink_buf;
-};
-
-constexpr int kMaxVarlenSeqs = 256;     // sequences per variable-length launch
 
 template <int D>
 struct PrefillCfg {
@@ -125,180 +85,6 @@ struct PrefillCfg {
 };
 
 // Which query rows and key tiles one work unit covers.
-struct UnitPlan {
-    int b, g, pair, qb;
-    int h0;          // query head of the unit's first head slot
-    int q0;          // first query row (relative to the q tensor)
-    int s0;          // absolute position of query row 0 of the sequence (chunk start, or 0)
-    int qs;          // s0 mod W (slot the next position would take)
-    int act1;        // second query head of the pair exists
-    int nc1, c1;     // cache run 1: tiles c1 .. c1+nc1-1
-    int nc2, c2;     // cache run 2
-    int nm, m0;      // main tiles m0 .. m0+nm-1
-    int sink_tile;   // sink tiles visited first: main tiles below the band (one-shot) or
-                     // sink-buffer tiles (chunk mode)
-    int n;           // total tiles
-    int nq;          // query rows of this sequence (== rows of its main k/v)
-    int row0;        // first packed row of this sequence in q/k/v (varlen), else 0
-    int tb;          // TMA batch coordinate of q/k/v (0 when packed)
-    size_t orow0;    // output row of query row 0 of this sequence
-};
-
-// Rows of sequence b of a packed batch: cu_seqlens[b+1] - cu_seqlens[b] when
-// 0 <= cu[b] <= cu[b+1] <= total rows, else 0 (a malformed sequence is
-// skipped, so no row outside the packed tensors is ever read or written).
-__device__ __forceinline__ int varlen_rows(const PrefillParams &p, int b) {
-    const int c0 = __ldg(p.cu_seqlens + b), c1 = __ldg(p.cu_seqlens + b + 1);
-    return (c0 >= 0 && c0 <= c1 && c1 <= p.Nq) ? c1 - c0 : 0;
-}
-
-// pre: shared-memory prefix sums of query blocks per sequence (varlen only).
-__device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, const int *pre) {
-    constexpr int BM = 128, BN = 128;
-    UnitPlan P;
-    int which = -1;
-    if (p.cu_seqlens) {
-        const int per = p.Hkv * p.npairs;
-        const int qbi = pre[p.B] - 1 - u / per;        // later blocks first
-        int r = u % per;
-        P.pair = r % p.npairs;
-        P.g = r / p.npairs;
-        int lo = 0, hi = p.B - 1;                       // last b with pre[b] <= qbi
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (pre[mid] <= qbi) lo = mid; else hi = mid - 1;
-        }
-        P.b = lo;
-        P.qb = qbi - pre[lo];
-        const int c0 = __ldg(p.cu_seqlens + lo);
-        P.nq = varlen_rows(p, lo);
-        P.row0 = P.nq > 0 ? c0 : 0;
-        P.tb = 0;
-        P.orow0 = (size_t)c0;
-    } else {
-        int pu = u;                          // pair unit; which: head of a split unit
-        if (u >= p.split_from) {
-            pu = p.split_from + (u - p.split_from) / 2;
-            which = (u - p.split_from) & 1;
-        }
-        const int per = p.B * p.Hkv * p.npairs;
-        P.qb = p.nqb - 1 - pu / per;         // latest (heaviest) query blocks first
-        int r = pu % per;
-        P.pair = r % p.npairs;
-        r /= p.npairs;
-        P.g = r % p.Hkv;
-        P.b = r / p.Hkv;
-        P.nq = p.Nq;
-        P.row0 = 0;
-        P.tb = P.b;
-        P.orow0 = (size_t)P.b * p.Nq;
-    }
-    const int span = p.qpair ? 2 * BM : BM;          // query rows of the unit
-    P.q0 = P.qb * span;
-    if (p.qpair) {
-        P.act1 = P.q0 + BM < P.nq;                   // the second block exists
-        P.h0 = P.g * p.G + P.pair;                   // one head per unit (npairs = G)
-    } else {
-        P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
-        P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
-    }
-    P.nc1 = P.nc2 = 0;
-    P.c1 = P.c2 = 0;
-    if (!p.chunk_mode) {
-        P.s0 = 0;
-        P.qs = 0;
-        const int lo = max(0, P.q0 - p.W + 1);
-        const int hi = min(P.nq - 1, P.q0 + span - 1);
-        P.m0 = lo / BN;
-        P.nm = hi / BN - P.m0 + 1;
-        // sink positions below the band live in the first ceil(S/128) tiles
-        P.sink_tile = min((p.sinks + BN - 1) / BN, P.m0);
-    } else {
-        P.s0 = __ldg(p.start_pos + P.b);
-        if (P.s0 < 0) {                       // invalid start: record it, attend as if 0
-            record_status(kStatusInvalid);
-            P.s0 = 0;
-        }
-        // sink positions j <= i - W exist for some row i of the block
-        P.sink_tile = (p.sink_buf > 0 && (long long)P.s0 + P.q0 + span - 1 >= p.W) ? (p.sink_buf + BN - 1) / BN : 0;
-        P.qs = P.s0 % p.W;
-        // oldest age any row of the block still needs: age < W - q0, age <= s0
-        const int A = min(p.W - P.q0 - 1, P.s0);
-        if (A >= 1) {
-            int last1 = -1;
-            if (P.qs >= 1) {                       // slots qs-A .. qs-1 (clipped at 0)
-                const int lo1 = max(0, P.qs - A);
-                P.c1 = lo1 / BN;
-                last1 = (P.qs - 1) / BN;
-                P.nc1 = last1 - P.c1 + 1;
-            }
-            if (A > P.qs) {                        // wrapped part: slots W-(A-qs) .. W-1
-                int lo2t = (p.W - (A - P.qs)) / BN;
-                if (lo2t <= last1) lo2t = last1 + 1;
-                const int hi2t = (p.W - 1) / BN;
-                if (lo2t <= hi2t) {
-                    P.c2 = lo2t;
-                    P.nc2 = hi2t - lo2t + 1;
-                }
-            }
-        }
-        const int lo = max(0, P.q0 - p.W + 1);          // chunks longer than W
-        const int hi = min(P.nq - 1, P.q0 + span - 1);
-        P.m0 = lo / BN;
-        P.nm = hi / BN - P.m0 + 1;
-    }
-    P.n = P.sink_tile + P.nc1 + P.nc2 + P.nm;
-    return P;
-}
-
-// Unit taken by CTA c of C in round k: rounds alternate direction, so the
-// CTAs that drew the heavier units of one round draw the lighter ones of the
-// next (units are ordered heaviest first), which evens out the per-CTA work;
-// >= the unit count once the CTA has no more work.
-__device__ __forceinline__ int unit_of(int k, int c, int C) {
-    return k * C + ((k & 1) ? (C - 1 - c) : c);
-}
-
-// Key tile j of a unit: source (1 = cache), first row (slot or key index),
-// and whether any element of the 128x128 tile may be masked.
-struct TileRef {
-    int cache;       // 0: main k/v, 1: rolling-buffer cache, 2: sink buffer (chunk mode)
-    int row0;
-    int masked;
-};
-
-__device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPlan &P, int j) {
-    constexpr int BM = 128, BN = 128;
-    const int span = p.qpair ? 2 * BM : BM;          // query rows of the unit
-    TileRef t;
-    if (j < P.sink_tile) {                  // only the sink positions of this tile count
-        t.cache = p.chunk_mode ? 2 : 0;
-        t.row0 = j * BN;
-        t.masked = 1;
-        return t;
-    }
-    j -= P.sink_tile;
-    if (j < P.nc1 + P.nc2) {
-        t.cache = 1;
-        const int tile = (j < P.nc1) ? (P.c1 + j) : (P.c2 + (j - P.nc1));
-        const int k0 = tile * BN;
-        t.row0 = k0;
-        const int t_last = min(P.q0 + span - 1, P.nq - 1);
-        const bool has_qs = (k0 <= P.qs) && (P.qs < k0 + BN);
-        const int max_age = (k0 + BN - 1 < P.qs) ? (P.qs - k0) : (p.W - (k0 - P.qs));
-        const bool clean = !has_qs && (k0 + BN <= p.W) && (max_age < p.W - t_last) &&
-                           (max_age <= P.s0);
-        t.masked = !clean;
-    } else {
-        t.cache = 0;
-        const int k0 = (P.m0 + (j - P.nc1 - P.nc2)) * BN;
-        t.row0 = k0;
-        const bool clean = (k0 + BN - 1 <= P.q0) && (k0 > P.q0 + span - 1 - p.W) && (k0 + BN <= P.nq);
-        t.masked = !clean;
-    }
-    return t;
-}
-
 // Rotary embedding of row `row` of a K-major, 128-byte-swizzled bf16 tile in
 // shared memory (the layout TMA writes): 16-byte chunk c of the row in a
 // 64-column region sits at chunk c ^ (row mod 8).
@@ -386,19 +172,10 @@ swa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         *abort_flag = 0;
         mbar_init_fence();
         if (p.cu_seqlens) {
-            // query blocks per sequence, prefix-summed (empty or malformed
-            // sequences count as empty; malformed ones are recorded; with
-            // skip_len1, sequences of one row too)
-            int acc = 0;
-            for (int b = 0; b < p.B; ++b) {
-                pre[b] = acc;
-                int n = varlen_rows(p, b);
-                if (n == 0 && __ldg(p.cu_seqlens + b + 1) != __ldg(p.cu_seqlens + b)) record_status(kStatusInvalid);
-                if (n == 1 && p.skip_len1) n = 0;
-                acc += (n + 127) / 128;
-            }
-            pre[p.B] = acc;
-            *unit_count = acc * p.Hkv * p.npairs;
+            // query blocks per sequence, prefix-summed (malformed sequences
+            // count as empty and are recorded)
+            if (varlen_prefix(p, pre)) record_status(kStatusInvalid);
+            *unit_count = pre[p.B] * p.Hkv * p.npairs;
         } else {
             *unit_count = p.num_units;
         }

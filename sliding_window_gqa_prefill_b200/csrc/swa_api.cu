@@ -133,37 +133,6 @@ bool bad_scale(float s) { return !(std::isfinite(s) && s > 0.f); }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// An odd group leaves the second head slot of its last pair unit empty (all
-// of them for G = 1); with a fixed-length batch of at least two waves of
-// units, a unit takes two consecutive 128-row query blocks of one head
-// instead (they share most key tiles), which keeps both softmax warpgroups
-// busy (B=2, N=16K, W=4K: G=3 867 -> 1000, G=5 866 -> 995, G=7 854 -> 957
-// TFLOP/s).  Even groups keep the pairs of heads, which also share each key
-// tile between the two heads.
-bool use_qpair(int G, bool varlen, long long units, int sms) {
-    return G % 2 == 1 && !varlen && units >= 2LL * sms;
-}
-
-// Chunk attention units (all about the same cost) fill whole waves of CTAs
-// except the last; when that wave is at most half full, its pair units are
-// split into two single-head units each, which fit in it and take about three
-// quarters of a pair unit's time (all of them when the whole launch is at
-// most half a wave).  Returns the first split pair unit and raises units by
-// the number split.
-int split_units(int &units, int G, int sms) {
-    if (G % 2 != 0 || units > 0x7fffffff - sms) return units;
-    if (2 * units <= sms) {           // a launch of at most half a wave: split every unit
-        units *= 2;
-        return 0;
-    }
-    if (units <= sms) return units;
-    const int rem = units % sms;
-    if (rem == 0 || 2 * rem > sms) return units;
-    const int from = units - rem;
-    units += rem;
-    return from;
-}
-
 template <int D>
 // mks / mvs: sink-buffer maps (chunk mode with sinks), else any valid map.
 swa_status_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
@@ -431,31 +400,8 @@ swa_status_t prefill_impl(const void *q, const void *k, const void *v, void *out
     if (swa_status_t e = make_operand_map(&mv, v, D, Hkv, N, mb)) return e;
 
     swa::PrefillParams p{};
-    p.B = B;
-    p.Nq = N;
-    p.Nk = N;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.G = G;
-    p.W = (int)Weff;
-    p.npairs = (G + 1) / 2;
-    p.nqb = (int)nqb;
-    p.num_units = (int)units;
-    if (use_qpair(G, cu_seqlens != nullptr, units, dev->sms)) {
-        p.qpair = 1;
-        p.npairs = G;
-        p.nqb = (int)((nqb + 1) / 2);
-        p.num_units = B * Hkv * G * p.nqb;
-    }
-    // the lightest blocks come last, so a full launch is not split; one of at
-    // most half a wave runs as single-head units
-    p.split_from = cu_seqlens ? 0x7fffffff : p.num_units;
-    if (!cu_seqlens && G % 2 == 0 && 2 * units <= dev->sms) {
-        p.split_from = 0;
-        p.num_units = (int)units * 2;
-    }
+    swa::prefill_units(p, B, N, Hq, Hkv, (int)Weff, cu_seqlens != nullptr, false, dev->sms);
     p.scale_log2 = scale * kLog2e;
-    p.chunk_mode = 0;
     p.start_pos = nullptr;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
@@ -505,25 +451,8 @@ swa_status_t prefill_chunk_impl(const void *q, const void *k, const void *v, voi
     if (swa_status_t e = make_operand_map(&mvc, v_cache, D, Hkv, W, B)) return e;
 
     swa::PrefillParams p{};
-    p.B = B;
-    p.Nq = C;
-    p.Nk = C;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.G = G;
-    p.W = W;
-    p.npairs = (G + 1) / 2;
-    p.nqb = (int)nqb;
-    p.num_units = (int)units;
-    if (use_qpair(G, cu_seqlens != nullptr, units, dev->sms)) {
-        p.qpair = 1;
-        p.npairs = G;
-        p.nqb = (int)((nqb + 1) / 2);
-        p.num_units = B * Hkv * G * p.nqb;
-    }
-    p.split_from = cu_seqlens ? 0x7fffffff : split_units(p.num_units, G, dev->sms);
+    swa::prefill_units(p, B, C, Hq, Hkv, W, cu_seqlens != nullptr, true, dev->sms);
     p.scale_log2 = scale * kLog2e;
-    p.chunk_mode = 1;
     p.start_pos = start_pos;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
