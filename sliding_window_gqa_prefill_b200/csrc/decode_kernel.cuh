@@ -22,7 +22,8 @@
 //    S = Q K^T for 16 keys is 2 x D/16 MMAs with K fed by ldmatrix, and
 //    O += P V is D/8 MMAs with V fed by ldmatrix.trans.  The S accumulator
 //    of a thread is exactly its A fragment of P (head = row, keys = columns),
-//    so P never leaves registers.  About 4 warp instructions per key row.
+//    so P never leaves registers.  About 23 warp instructions per key row
+//    of one KV head, the copies and the split's merge included.
 //  * online softmax per head in base 2, scale applied to S in fp32; the
 //    exponent offset of a head is raised (exact maximum over the block,
 //    rescale of l and o) only when a score exceeds it by more than 2^8, so
