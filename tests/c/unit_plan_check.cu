@@ -3,6 +3,8 @@
 //
 // For each case the launch parameters come from prefill_units() as the host
 // API fills them, and every unit of the launch is planned.  Checked:
+//  * the persistent blocks (min(units, SMs) of them, alternating direction
+//    every round) take every unit exactly once;
 //  * every (sequence, query head, query row) is computed by exactly one head
 //    slot of one unit, and that head belongs to the unit's KV head
 //    (contiguous groups: head h uses KV head h / G);
@@ -77,6 +79,17 @@ bool check(const Case &c0) {
         if (swa::varlen_prefix(p, pre.data())) return fail(c, "malformed offsets reported");
         units = pre[c.B] * p.Hkv * p.npairs;
         if (units > p.num_units) return fail(c, "packed units above the host's bound", units, p.num_units);
+    }
+
+    // the persistent schedule: over the alternating rounds, the grid's blocks
+    // take every unit exactly once
+    {
+        const int C = units < c.sms ? units : c.sms;
+        std::vector<int> taken(units, 0);
+        for (int cta = 0; cta < C; ++cta)
+            for (int k = 0, u; (u = swa::unit_of(k, cta, C)) < units; ++k) ++taken[u];
+        for (int u = 0; u < units; ++u)
+            if (taken[u] != 1) return fail(c, "unit not taken exactly once", u, taken[u], C);
     }
 
     // rows per sequence

@@ -3,7 +3,8 @@ compiles the planner the kernel's warps call (prefill_plan.cuh) for the host
 and enumerates every unit of 30 launches (one-shot, query-block pairs for odd
 groups, chunk mode through the rolling buffer, sinks, packed batches, the
 last-wave and half-wave single-head splits, windows whose edge falls on a
-tile's first key).  Each query row of each head must be computed exactly once,
+tile's first key).  The persistent blocks must take every unit exactly once,
+each query row of each head must be computed exactly once,
 by a unit of its KV head, and the unit's key tiles must hold exactly the row's
 keys (window, sinks, buffer slots), tiles marked clean needing no mask."""
 import os
