@@ -55,10 +55,11 @@ struct PrefillParams {
     // variable-length batch: q/k/v/out packed as [total, H, D]; sequence b is
     // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (null: fixed-length [B, N, H, D])
     const int32_t *cu_seqlens;
-    // 1 (odd group of heads, fixed-length): the two head slots of
-    // a unit are two consecutive 128-row query blocks of one head, which share
-    // the key tiles of their bands, instead of two heads of the group; npairs
-    // is then G (one head per unit) and nqb counts the 256-row pairs
+    // 1 (odd group of heads): the two head slots of a unit are two
+    // consecutive 128-row query blocks of one head, which share the key tiles
+    // of their bands, instead of two heads of the group; npairs is then G (one
+    // head per unit) and nqb counts the 256-row pairs (a packed batch's
+    // prefix sums count them per sequence)
     int qpair;
     // variable-length chunk batch: 1 leaves sequences of one row to the
     // decode kernel (no work units for them)
@@ -248,10 +249,12 @@ __host__ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, con
     return t;
 }
 
-// Query blocks per sequence of a packed batch, prefix-summed into
-// pre[0..B] (empty or malformed sequences count as empty, as do sequences of
-// one row with skip_len1).  Returns true if a malformed sequence was seen.
+// Query blocks (pairs of blocks with qpair) per sequence of a packed batch,
+// prefix-summed into pre[0..B] (empty or malformed sequences count as empty,
+// as do sequences of one row with skip_len1).  Returns true if a malformed
+// sequence was seen.
 __host__ __device__ __forceinline__ bool varlen_prefix(const PrefillParams &p, int *pre) {
+    const int rows = p.qpair ? 256 : 128;
     int acc = 0;
     bool bad = false;
     for (int b = 0; b < p.B; ++b) {
@@ -259,7 +262,7 @@ __host__ __device__ __forceinline__ bool varlen_prefix(const PrefillParams &p, i
         int n = varlen_rows(p, b);
         if (n == 0 && ld_i32(p.cu_seqlens + b + 1) != ld_i32(p.cu_seqlens + b)) bad = true;
         if (n == 1 && p.skip_len1) n = 0;
-        acc += (n + 127) / 128;
+        acc += (n + rows - 1) / rows;
     }
     pre[p.B] = acc;
     return bad;
@@ -268,14 +271,15 @@ __host__ __device__ __forceinline__ bool varlen_prefix(const PrefillParams &p, i
 // ------------------------------------------------------------------ host side
 
 // An odd group leaves the second head slot of its last pair unit empty (all
-// of them for G = 1); with a fixed-length batch of at least two waves of
-// units, a unit takes two consecutive 128-row query blocks of one head
+// of them for G = 1); with at least two waves of units (for a packed batch,
+// by the host's upper bound), a unit takes two consecutive 128-row query
+// blocks of one head
 // instead (they share most key tiles), which keeps both softmax warpgroups
 // busy (B=2, N=16K, W=4K: G=3 867 -> 1000, G=5 866 -> 995, G=7 854 -> 957
 // TFLOP/s).  Even groups keep the pairs of heads, which also share each key
 // tile between the two heads.
-inline bool use_qpair(int G, bool varlen, long long units, int sms) {
-    return G % 2 == 1 && !varlen && units >= 2LL * sms;
+inline bool use_qpair(int G, long long units, int sms) {
+    return G % 2 == 1 && units >= 2LL * sms;
 }
 
 // Chunk attention units (all about the same cost) fill whole waves of CTAs
@@ -322,11 +326,13 @@ inline void prefill_units(PrefillParams &p, int B, int Nq, int Hq, int Hkv, int 
     p.nqb = (int)nqb;
     p.num_units = (int)units;
     p.qpair = 0;
-    if (use_qpair(G, varlen, units, sms)) {
+    if (use_qpair(G, units, sms)) {
+        // pairs of query blocks: a packed sequence of n rows takes
+        // ceil(n / 256) of them, at most N / 256 + 1
         p.qpair = 1;
         p.npairs = G;
         p.nqb = (int)((nqb + 1) / 2);
-        p.num_units = B * Hkv * G * p.nqb;
+        p.num_units = (int)(varlen ? (long long)Hkv * G * (p.nqb + B) : (long long)B * Hkv * G * p.nqb);
     }
     p.chunk_mode = chunk ? 1 : 0;
     if (varlen) {

@@ -215,6 +215,12 @@ int main() {
         {"varlen chunk", 5, 900, 8, 2, 512, true, 0, {0, 3000, 7, 512, 100}, {0, 300, 301, 600, 600, 900}, false, sms},
         {"varlen chunk, one-row sequences to decode", 5, 900, 8, 2, 512, true, 0, {0, 3000, 7, 512, 100},
          {0, 300, 301, 600, 601, 900}, true, sms},
+        // packed batches in pairs of query blocks (odd groups, two waves by the host's bound)
+        {"varlen qpair MHA", 4, 2500, 32, 32, 500, false, 0, {}, {0, 700, 1300, 1301, 2500}, false, sms},
+        {"varlen qpair G=3 W=383", 3, 2300, 24, 8, 383, false, 0, {}, {0, 1000, 1001, 2300}, false, sms},
+        {"varlen chunk qpair G=3", 3, 2300, 24, 8, 1024, true, 0, {0, 5000, 100}, {0, 1000, 1001, 2300}, false, sms},
+        {"varlen chunk qpair G=3, one-row sequences to decode", 4, 2300, 24, 8, 1024, true, 0, {0, 5000, 100, 9},
+         {0, 1000, 1001, 2299, 2300}, true, sms},
     };
     for (const Case &c : cases)
         if (!check(c)) return 1;

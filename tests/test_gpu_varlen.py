@@ -38,7 +38,10 @@ def close(got, ref, what):
 
 
 @pytest.mark.parametrize("lens,Hq,Hkv,D,W", [([300, 1, 0, 1000, 129], 8, 2, 128, 256),
-                                            ([64, 700, 5], 6, 2, 64, 100)])
+                                            ([64, 700, 5], 6, 2, 64, 100),
+                                            # odd groups at two waves of units: pairs of query blocks
+                                            ([700, 600, 1, 1200], 32, 32, 128, 500),
+                                            ([1000, 1, 1299], 24, 8, 64, 383)])
 def test_prefill_varlen_matches_per_sequence_oracle(oracle_mod, lens, Hq, Hkv, D, W):
     total = sum(lens)
     cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
@@ -105,6 +108,18 @@ def _mixed(oracle_mod, hist, now, Hq, Hkv, D, W, seed):
 def test_mixed_chunks_and_decode_in_one_launch(oracle_mod, Hq, Hkv):
     # per sequence: history length already in the buffer, tokens in this call
     _mixed(oracle_mod, [1000, 7000, 0, 300, 50], [500, 1, 300, 0, 1], Hq, Hkv, 128, 256, 90)
+
+
+@pytest.mark.parametrize("Hq,Hkv,hist,now", [
+    (24, 8, [0, 5000, 100, 9], [1000, 1, 1298, 1]),      # groups of 3, 352 head-pair units: block pairs
+    (32, 32, [2000, 0, 7], [800, 900, 1]),               # one head per KV head
+])
+def test_mixed_batch_in_pairs_of_query_blocks(oracle_mod, Hq, Hkv, hist, now):
+    """A packed chunk batch with an odd group and at least two waves of units
+    takes units of two consecutive query blocks of one head (prefix sums of
+    256-row pairs per sequence); its one-row sequences still go to the decode
+    kernel."""
+    _mixed(oracle_mod, hist, now, Hq, Hkv, 128, 1024, 95)
 
 
 @pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8, 12])
