@@ -81,7 +81,7 @@ struct UnitPlan {
     int q0;          // first query row (relative to the q tensor)
     int s0;          // absolute position of query row 0 of the sequence (chunk start, or 0)
     int qs;          // s0 mod W (slot the next position would take)
-    int act1;        // second query head of the pair exists
+    int act1;        // second query head (or block) of the pair exists
     int nc1, c1;     // cache run 1: tiles c1 .. c1+nc1-1
     int nc2, c2;     // cache run 2
     int nm, m0;      // main tiles m0 .. m0+nm-1
@@ -100,6 +100,14 @@ struct UnitPlan {
 __host__ __device__ __forceinline__ int varlen_rows(const PrefillParams &p, int b) {
     const int c0 = ld_i32(p.cu_seqlens + b), c1 = ld_i32(p.cu_seqlens + b + 1);
     return (c0 >= 0 && c0 <= c1 && c1 <= p.Nq) ? c1 - c0 : 0;
+}
+
+// Query rows whose key tiles a unit visits, from q0: 256 for a pair of query
+// blocks whose second block exists, else 128 (a head pair, a split pair, or
+// a pair whose second block lies past the sequence, whose rows all sit
+// below q0 + 128).
+__host__ __device__ __forceinline__ int unit_span(const PrefillParams &p, const UnitPlan &P) {
+    return (p.qpair && P.act1) ? 256 : 128;
 }
 
 // pre: shared-memory prefix sums of query blocks per sequence (varlen only).
@@ -126,7 +134,7 @@ __host__ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, i
         P.tb = 0;
         P.orow0 = (size_t)c0;
     } else {
-        int pu = u;                          // pair unit; which: head of a split unit
+        int pu = u;                          // pair unit; which: head (or block) of a split unit
         if (u >= p.split_from) {
             pu = p.split_from + (u - p.split_from) / 2;
             which = (u - p.split_from) & 1;
@@ -143,15 +151,18 @@ __host__ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, i
         P.tb = P.b;
         P.orow0 = (size_t)P.b * p.Nq;
     }
-    const int span = p.qpair ? 2 * BM : BM;          // query rows of the unit
-    P.q0 = P.qb * span;
+    P.q0 = P.qb * (p.qpair ? 2 * BM : BM);
     if (p.qpair) {
-        P.act1 = P.q0 + BM < P.nq;                   // the second block exists
         P.h0 = P.g * p.G + P.pair;                   // one head per unit (npairs = G)
+        // a split pair is one of its two blocks; else the second block exists
+        // unless the sequence ends in the first
+        if (which > 0) P.q0 += BM;
+        P.act1 = which < 0 && P.q0 + BM < P.nq;
     } else {
         P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
         P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
     }
+    const int span = unit_span(p, P);
     P.nc1 = P.nc2 = 0;
     P.c1 = P.c2 = 0;
     if (!p.chunk_mode) {
@@ -218,8 +229,11 @@ struct TileRef {
 };
 
 __host__ __device__ __forceinline__ TileRef tile_ref(const PrefillParams &p, const UnitPlan &P, int j) {
-    constexpr int BM = 128, BN = 128;
-    const int span = p.qpair ? 2 * BM : BM;          // query rows of the unit
+    constexpr int BN = 128;
+    // rows over which a tile is tested clean: both blocks of a pair, also
+    // for a split pair (a superset of its rows, so the test stays exact)
+    // -- a constant of the launch, so the softmax loop holds no extra state
+    const int span = p.qpair ? 2 * BN : BN;
     TileRef t;
     if (j < P.sink_tile) {                  // only the sink positions of this tile count
         t.cache = p.chunk_mode ? 2 : 0;
@@ -288,8 +302,8 @@ inline bool use_qpair(int G, long long units, int sms) {
 // quarters of a pair unit's time (all of them when the whole launch is at
 // most half a wave).  Returns the first split pair unit and raises units by
 // the number split.
-inline int split_units(int &units, int G, int sms) {
-    if (G % 2 != 0 || units > 0x7fffffff - sms) return units;
+inline int split_units(int &units, bool splittable, int sms) {
+    if (!splittable || units > 0x7fffffff - sms) return units;
     if (2 * units <= sms) {           // a launch of at most half a wave: split every unit
         units *= 2;
         return 0;
@@ -338,7 +352,19 @@ inline void prefill_units(PrefillParams &p, int B, int Nq, int Hq, int Hkv, int 
     if (varlen) {
         p.split_from = 0x7fffffff;
     } else if (chunk) {
-        p.split_from = split_units(p.num_units, G, sms);
+        // head pairs of an even group split into their two heads; pairs of
+        // query blocks into their two blocks, unless a pair with one block
+        // (the sequence's last, when Nq is not a multiple of 256) would be
+        // among them
+        int n = p.num_units;
+        const int from = split_units(n, G % 2 == 0 || p.qpair, sms);
+        const bool one_block_pair = p.qpair && Nq % 256 != 0 && from < B * Hkv * G;
+        if (!one_block_pair) {
+            p.split_from = from;
+            p.num_units = n;
+        } else {
+            p.split_from = p.num_units;
+        }
     } else {
         // the lightest blocks come last, so a full launch is not split; one of
         // at most half a wave runs as single-head units

@@ -210,6 +210,12 @@ int main() {
         {"chunk 4096 last-wave split", 1, 4096, 32, 8, 4096, true, 0, {12288}, {}, false, sms},
         {"chunk qpair G=3", 2, 1280, 24, 8, 1280, true, 0, {1280, 2560}, {}, false, sms},
         {"chunk qpair MHA sinks", 1, 1280, 32, 32, 1280, true, 130, {1280}, {}, false, sms},
+        // pairs of query blocks split into their blocks in a short last wave
+        {"chunk qpair MHA 4096 last-wave split", 1, 4096, 32, 32, 4096, true, 0, {12288}, {}, false, sms},
+        {"chunk qpair ragged, split away from the one-block pairs", 1, 1000, 40, 40, 1000, true, 4, {2000}, {}, false,
+         sms},
+        {"chunk qpair one-block pairs in the last wave: no split", 1, 200, 300, 300, 256, true, 0, {1000}, {}, false,
+         sms},
         // packed batches
         {"varlen one-shot", 6, 1000, 32, 8, 256, false, 0, {}, {0, 1, 129, 130, 700, 700, 1000}, false, sms},
         {"varlen chunk", 5, 900, 8, 2, 512, true, 0, {0, 3000, 7, 512, 100}, {0, 300, 301, 600, 600, 900}, false, sms},
