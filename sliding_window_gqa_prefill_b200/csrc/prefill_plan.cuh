@@ -64,6 +64,10 @@ struct PrefillParams {
     // variable-length chunk batch: 1 leaves sequences of one row to the
     // decode kernel (no work units for them)
     int skip_len1;
+    // 1 (odd group, a launch whose single-head units all fit in one wave):
+    // every unit is one query head of the group (npairs = G) and one 128-row
+    // block, so the SMs a pair launch would leave idle take the second heads
+    int single;
     // attention sinks (one-shot prefill): positions j < sinks stay visible to
     // every query besides its window
     int sinks;
@@ -159,8 +163,10 @@ __host__ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, i
         if (which > 0) P.q0 += BM;
         P.act1 = which < 0 && P.q0 + BM < P.nq;
     } else {
-        P.act1 = which < 0 && (2 * P.pair + 1) < p.G;
-        P.h0 = P.g * p.G + 2 * P.pair + (which > 0 ? 1 : 0);
+        // head pairs (a split pair: one of its heads); single: one head per
+        // unit (npairs = G)
+        P.act1 = !p.single && which < 0 && (2 * P.pair + 1) < p.G;
+        P.h0 = P.g * p.G + (p.single ? P.pair : 2 * P.pair + (which > 0 ? 1 : 0));
     }
     const int span = unit_span(p, P);
     P.nc1 = P.nc2 = 0;
@@ -340,6 +346,7 @@ inline void prefill_units(PrefillParams &p, int B, int Nq, int Hq, int Hkv, int 
     p.nqb = (int)nqb;
     p.num_units = (int)units;
     p.qpair = 0;
+    p.single = 0;
     if (use_qpair(G, units, sms)) {
         // pairs of query blocks: a packed sequence of n rows takes
         // ceil(n / 256) of them, at most N / 256 + 1
@@ -367,11 +374,17 @@ inline void prefill_units(PrefillParams &p, int B, int Nq, int Hq, int Hkv, int 
         }
     } else {
         // the lightest blocks come last, so a full launch is not split; one of
-        // at most half a wave runs as single-head units
+        // at most half a wave runs as single-head units (an odd group's pairs
+        // cannot be split in two, so its units are then the heads themselves)
         p.split_from = p.num_units;
         if (G % 2 == 0 && 2 * units <= sms) {
             p.split_from = 0;
             p.num_units = (int)units * 2;
+        } else if (G % 2 == 1 && G > 1 && !p.qpair && (long long)B * Hkv * G * nqb <= sms) {
+            p.single = 1;
+            p.npairs = G;
+            p.num_units = B * Hkv * G * (int)nqb;
+            p.split_from = p.num_units;
         }
     }
 }

@@ -185,6 +185,10 @@ int main() {
         {"one-shot odd group 6/2 below two waves", 1, 900, 6, 2, 256, false, 0, {}, {}, false, sms},
         {"one-shot G=3 head pairs, 288 units", 1, 2304, 24, 8, 600, false, 0, {}, {}, false, sms},
         {"one-shot half-wave split 32/8", 1, 256, 32, 8, 64, false, 0, {}, {}, false, sms},
+        // odd groups in one wave: one head per unit
+        {"one-shot single heads G=7", 1, 512, 28, 4, 256, false, 0, {}, {}, false, sms},
+        {"one-shot single heads G=3 sinks", 2, 300, 6, 2, 100, false, 4, {}, {}, false, sms},
+        {"one-shot G=3 past one wave of single heads", 1, 1024, 24, 8, 383, false, 0, {}, {}, false, sms},
         {"one-shot W=1", 1, 300, 4, 2, 1, false, 0, {}, {}, false, sms},
         // windows of 128k-1 keys: a tile's first key lands on the last row's window edge
         {"one-shot W=255", 2, 1000, 8, 2, 255, false, 0, {}, {}, false, sms},
