@@ -114,7 +114,8 @@ __host__ __device__ __forceinline__ int unit_span(const PrefillParams &p, const 
     return (p.qpair && P.act1) ? 256 : 128;
 }
 
-// pre: shared-memory prefix sums of query blocks per sequence (varlen only).
+// pre: prefix sums of query blocks (pairs of blocks with qpair) per sequence
+// (packed batches only; varlen_prefix).
 __host__ __device__ __forceinline__ UnitPlan plan_unit(const PrefillParams &p, int u, const int *pre) {
     constexpr int BM = 128, BN = 128;
     UnitPlan P;
