@@ -27,7 +27,9 @@
 // rule slot = p mod W ("Rolling Buffer KV Cache 동작 설명"), and the attention
 // sinks of the aionda.blog page (the first few positions kept).
 //
-// Prints "ok <cases> <rows>" and exits 0, or the first mismatch and exits 1.
+// Also 160 seeded random launches (shapes, windows, sinks, packed offsets,
+// buffer positions and SM counts drawn).  Prints "ok <cases> <rows>" and
+// exits 0, or the first mismatch and exits 1.
 #include <cstdio>
 #include <cstdlib>
 #include <set>
@@ -234,6 +236,53 @@ int main() {
     };
     for (const Case &c : cases)
         if (!check(c)) return 1;
-    std::printf("ok %zu %lld\n", cases.size(), g_rows);
+
+    // seeded random launches; small SM counts make the two-wave, last-wave
+    // and one-wave policies trigger at small sizes
+    unsigned long long state = 0x2545F4914F6CDD1DULL;
+    auto draw = [&](int lo, int hi) {               // uniform on [lo, hi]
+        state ^= state << 13;
+        state ^= state >> 7;
+        state ^= state << 17;
+        return lo + (int)(state % (unsigned long long)(hi - lo + 1));
+    };
+    const int sm_choices[] = {148, 33, 16, 8, 3};
+    int random_cases = 0;
+    for (int it = 0; it < 160; ++it) {
+        Case c;
+        c.name = "random";
+        const int mode = draw(0, 3);                // one-shot, chunk, packed one-shot, packed chunk
+        c.Hkv = draw(1, 2);
+        c.Hq = c.Hkv * draw(1, 8);
+        c.W = draw(1, 600);
+        c.sms = sm_choices[draw(0, 4)];
+        c.chunk = mode == 1 || mode == 3;
+        c.skip_len1 = false;
+        c.S = 0;
+        if (mode == 0 || mode == 1) {
+            c.B = draw(1, 2);
+            c.N = c.chunk ? draw(1, c.W < 500 ? c.W : 500) : draw(1, 500);
+            if (draw(0, 2) == 0) c.S = draw(1, 140);     // sinks (fixed-length calls only)
+        } else {
+            c.B = draw(1, 4);
+            c.cu.push_back(0);
+            for (int b = 0; b < c.B; ++b) {
+                const int kind = draw(0, 4);
+                c.cu.push_back(c.cu.back() + (kind == 0 ? 0 : kind == 1 ? 1 : draw(2, 300)));
+            }
+            c.N = c.cu.back();
+            if (c.N == 0) continue;                 // an empty packed call is rejected by the host
+            c.skip_len1 = c.chunk && draw(0, 1) == 1;
+        }
+        if (c.chunk)
+            for (int b = 0; b < c.B; ++b) c.start.push_back(draw(0, 3) == 0 ? 0 : draw(0, 4000));
+        if (!check(c)) {
+            std::printf("  (random case %d: B=%d N=%d Hq=%d Hkv=%d W=%d chunk=%d S=%d sms=%d)\n", it, c.B, c.N, c.Hq,
+                        c.Hkv, c.W, (int)c.chunk, c.S, c.sms);
+            return 1;
+        }
+        ++random_cases;
+    }
+    std::printf("ok %zu %lld (and %d random)\n", cases.size(), g_rows, random_cases);
     return 0;
 }

@@ -6,7 +6,9 @@ pairs and in query-block pairs, the
 last-wave and half-wave single-head splits, one head per unit for short
 odd-group launches, pairs of query blocks split into
 their blocks in a short last wave, windows whose edge falls on a
-tile's first key).  The persistent blocks must take every unit exactly once,
+tile's first key), then 160 seeded random launches whose SM count is drawn too
+(3 to 148 SMs, so every mode triggers at small sizes).  The persistent blocks
+must take every unit exactly once,
 each query row of each head must be computed exactly once,
 by a unit of its KV head, and the unit's key tiles must hold exactly the row's
 keys (window, sinks, buffer slots), tiles marked clean needing no mask."""
@@ -29,3 +31,4 @@ def test_every_row_once_and_exactly_its_keys(tmp_path):
     assert r.returncode == 0, r.stdout + r.stderr
     words = r.stdout.split()
     assert words[0] == "ok" and int(words[1]) == 40 and int(words[2]) > 1400000, r.stdout
+    assert words[3:5] == ["(and", "157"], r.stdout          # seeded random launches (3 empty ones skipped)
